@@ -1,0 +1,357 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against a closed form, a special case that reduces
+to a library routine, a brute-force enumeration, an invariant, or a worked
+example of the DSpark pages -- never against a retyped copy of its own loops.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy import special, stats
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bf16(a):
+    return synth.f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def _f(a):
+    return synth.bf16_bits_to_f32(a).astype(np.float64)
+
+
+def _tiny_draft_inputs(nb, gamma, V, r, w_std, seed):
+    rng = np.random.default_rng(seed)
+    W1 = _bf16(rng.normal(0, w_std, (V, r)))
+    W2 = _bf16(rng.normal(0, w_std, (r, V)))
+    U = _bf16(rng.normal(0, 1.0, (nb, gamma, V)))
+    anchor = rng.integers(0, V, nb).astype(np.int32)
+    return U, anchor, W1, W2
+
+
+# ---------------------------------------------------------------------------
+# Markov head (gdymind.com "DSpark", section 4): B = W1 W2 "in principle a full
+# V x V matrix" -- the low-rank path must equal drafting with the materialised
+# full transition matrix.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("V,r,gamma,nb", [(64, 8, 6, 3), (300, 16, 5, 4), (1000, 256, 3, 2)])
+def test_draft_equals_full_transition_matrix(oracle_mod, V, r, gamma, nb):
+    U, anchor, W1, W2 = _tiny_draft_inputs(nb, gamma, V, r, 0.6, seed=V)
+    Bfull = _f(W1) @ _f(W2)                      # [V, V] in fp64
+    x, logit, gap = oracle_mod.draft(U, anchor, W1, W2)
+    Uf = _f(U)
+    for i in range(nb):
+        prev = anchor[i]
+        for k in range(gamma):
+            l = Uf[i, k] + Bfull[prev]
+            xk = int(np.argmax(l))
+            assert x[i, k] == xk
+            assert logit[i, k] == pytest.approx(l[xk], abs=1e-10)
+            srt = np.sort(l)
+            assert gap[i, k] == pytest.approx(srt[-1] - srt[-2], abs=1e-10)
+            prev = xk
+    # the bias must actually move the choice somewhere in these cases
+    plain = np.argmax(Uf, axis=2)
+    assert (plain != x).any()
+
+
+def test_draft_zero_factor_is_parallel_argmax(oracle_mod):
+    V, r, gamma, nb = 500, 32, 7, 5
+    U, anchor, W1, W2 = _tiny_draft_inputs(nb, gamma, V, r, 0.5, seed=11)
+    for zero in ("W1", "W2"):
+        a = np.zeros_like(W1) if zero == "W1" else W1
+        b = np.zeros_like(W2) if zero == "W2" else W2
+        x, logit, _ = oracle_mod.draft(U, anchor, a, b)
+        np.testing.assert_array_equal(x, np.argmax(_f(U), axis=2))
+        np.testing.assert_array_equal(logit, np.max(_f(U), axis=2))
+
+
+def test_draft_ties_take_smallest_index(oracle_mod):
+    V, r, gamma = 64, 8, 4
+    U = np.zeros((1, gamma, V), dtype=np.uint16)
+    U[0, :, [5, 9, 40]] = _bf16([3.0])[0]
+    x, logit, gap = oracle_mod.draft(U, np.array([2], np.int32), np.zeros((V, r), np.uint16),
+                                     np.zeros((r, V), np.uint16))
+    assert (x == 5).all() and (logit == 3.0).all() and (gap == 0.0).all()
+
+
+def test_draft_rejects_bad_anchor(oracle_mod):
+    U, anchor, W1, W2 = _tiny_draft_inputs(1, 2, 64, 8, 0.1, seed=1)
+    with pytest.raises(ValueError):
+        oracle_mod.draft(U, np.array([64], np.int32), W1, W2)
+
+
+# ---------------------------------------------------------------------------
+# Gumbel-max: frequencies must follow softmax(l / tau)
+# ---------------------------------------------------------------------------
+def test_gumbel_max_frequencies_follow_softmax(oracle_mod):
+    V, r, gamma, nb, tau = 8, 4, 50, 2000, 0.7
+    l = np.array([0.0, 0.5, -1.0, 1.25, 0.25, -0.5, 1.0, 0.75], dtype=np.float32)
+    U = np.broadcast_to(_bf16(l), (nb, gamma, V)).copy()
+    W1 = np.zeros((V, r), np.uint16)
+    W2 = np.zeros((r, V), np.uint16)
+    x, logit, _ = oracle_mod.draft(U, np.zeros(nb, np.int32), W1, W2, mode=1, tau=tau, seed=1234)
+    counts = np.bincount(x.ravel(), minlength=V)
+    p = special.softmax(_f(_bf16(l)) / tau)
+    chi2, pval = stats.chisquare(counts, p * counts.sum())
+    assert pval > 1e-4, (counts, p * counts.sum(), pval)
+    # the reported logit is the unperturbed one at the chosen token
+    np.testing.assert_array_equal(logit, _f(_bf16(l))[x])
+
+
+def test_gumbel_small_temperature_is_greedy(oracle_mod):
+    V, r, gamma, nb = 200, 8, 6, 6
+    U, anchor, W1, W2 = _tiny_draft_inputs(nb, gamma, V, r, 0.3, seed=5)
+    xg, _, gapg = oracle_mod.draft(U, anchor, W1, W2, mode=0)
+    xs, _, _ = oracle_mod.draft(U, anchor, W1, W2, mode=1, tau=1e-6, seed=99)
+    # noise is at most about 17 in size, so with tau = 1e-6 only gaps below 4e-5 can flip
+    ok = gapg > 1e-4
+    assert ok.mean() > 0.9
+    np.testing.assert_array_equal(xg[ok], xs[ok])
+
+
+def test_noise_key_uses_request_position_and_vocab(oracle_mod):
+    g = {(b, k, v): oracle_mod.gumbel(7, b, k, v) for b in range(3) for k in (1, 2) for v in range(9)}
+    assert len(set(g.values())) == len(g)
+
+
+# ---------------------------------------------------------------------------
+# Philox4x32-10 (SC'11): each round is a bijection.  The inverse below undoes a
+# round with the published multipliers and Weyl constants; a wrong constant or
+# word wiring in the oracle breaks the round trip.  (Agreement with other
+# Philox implementations is not pinned: no known-answer vectors are at hand.)
+# ---------------------------------------------------------------------------
+_M0, _M1 = 0xD2511F53, 0xCD9E8D57
+_W0, _W1 = 0x9E3779B9, 0xBB67AE85
+_MASK = 0xFFFFFFFF
+
+
+def _philox_inverse(y, key):
+    keys = [((key[0] + i * _W0) & _MASK, (key[1] + i * _W1) & _MASK) for i in range(10)]
+    inv0, inv1 = pow(_M0, -1, 1 << 32), pow(_M1, -1, 1 << 32)
+    y0, y1, y2, y3 = (int(t) for t in y)
+    for k0, k1 in reversed(keys):
+        x2 = (y1 * inv1) & _MASK
+        x0 = (y3 * inv0) & _MASK
+        x1 = y0 ^ ((_M1 * x2) >> 32) ^ k0
+        x3 = y2 ^ ((_M0 * x0) >> 32) ^ k1
+        y0, y1, y2, y3 = x0, x1, x2, x3
+    return [y0, y1, y2, y3]
+
+
+def test_philox_rounds_invert(oracle_mod):
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        ctr = rng.integers(0, 2**32, 4, dtype=np.uint64).astype(np.uint32)
+        key = rng.integers(0, 2**32, 2, dtype=np.uint64).astype(np.uint32)
+        out = oracle_mod.philox4x32_10(ctr, key)
+        assert _philox_inverse(out, [int(k) for k in key]) == [int(c) for c in ctr]
+
+
+def test_philox_output_is_uniform(oracle_mod):
+    words = np.concatenate([oracle_mod.philox4x32_10([i, 0, 5, 0], [1, 2]) for i in range(4096)])
+    hist = np.bincount((words >> 28).astype(np.int64), minlength=16)
+    assert stats.chisquare(hist).pvalue > 1e-4
+
+
+def test_uniform_from_word_stays_inside_open_interval(oracle_mod):
+    assert oracle_mod.uniform_from_word(0) == 2.0**-24
+    assert oracle_mod.uniform_from_word(0xFFFFFFFF) == 1.0 - 2.0**-24
+    assert oracle_mod.uniform_from_word(1 << 31) == 0.5 + 2.0**-24
+
+
+# ---------------------------------------------------------------------------
+# Confidence head + Sequential Temperature Scaling + survival product
+# (gdymind.com "DSpark", section 5)
+# ---------------------------------------------------------------------------
+def _conf_inputs(B, gamma, d, r, V, seed):
+    rng = np.random.default_rng(seed)
+    h = _bf16(rng.normal(0, 1, (B, gamma, d)))
+    W1 = _bf16(rng.normal(0, 0.5, (V, r)))
+    w = _bf16(rng.normal(0, 1 / math.sqrt(d + r), d + r))
+    anchor = rng.integers(0, V, B).astype(np.int32)
+    x = rng.integers(0, V, (B, gamma)).astype(np.int32)
+    T = rng.uniform(1, 3, gamma).astype(np.float32)
+    return h, anchor, x, W1, w, T
+
+
+def test_confidence_one_hot_weights_select_inputs(oracle_mod):
+    B, gamma, d, r, V = 3, 5, 24, 8, 50
+    h, anchor, x, W1, w, T = _conf_inputs(B, gamma, d, r, V, 1)
+    ones = np.ones(gamma, np.float32)
+    hf, Ef = _f(h), _f(W1)
+    prev = np.concatenate([anchor[:, None], x[:, :-1]], axis=1)   # x_{k-1}, x_0 = anchor
+    for i in (0, 7, d - 1):
+        e = np.zeros(d + r, np.uint16); e[i] = _bf16([1.0])[0]
+        out = oracle_mod.confidence(h, anchor, x, W1, e, 0.25, ones)
+        np.testing.assert_allclose(out["z"], hf[:, :, i] + 0.25, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out["c"], special.expit(hf[:, :, i] + 0.25), rtol=1e-12)
+    for j in (0, 3, r - 1):
+        e = np.zeros(d + r, np.uint16); e[d + j] = _bf16([1.0])[0]
+        out = oracle_mod.confidence(h, anchor, x, W1, e, -0.5, ones)
+        np.testing.assert_allclose(out["z"], Ef[prev, j] - 0.5, rtol=0, atol=1e-12)
+
+
+def test_confidence_zero_weights_give_bias_only(oracle_mod):
+    B, gamma, d, r, V = 2, 6, 16, 8, 30
+    h, anchor, x, W1, w, T = _conf_inputs(B, gamma, d, r, V, 2)
+    out = oracle_mod.confidence(h, anchor, x, W1, np.zeros(d + r, np.uint16), 1.0, T)
+    np.testing.assert_allclose(out["c"], np.broadcast_to(special.expit(1.0 / T.astype(np.float64)),
+                                                         (B, gamma)), rtol=1e-13)
+
+
+def test_sts_temperature_scales_the_logit(oracle_mod):
+    B, gamma, d, r, V = 4, 7, 32, 16, 80
+    h, anchor, x, W1, w, T = _conf_inputs(B, gamma, d, r, V, 3)
+    c1 = oracle_mod.confidence(h, anchor, x, W1, w, 1.0, np.ones(gamma, np.float32))["c"]
+    cT = oracle_mod.confidence(h, anchor, x, W1, w, 1.0, T)["c"]
+    # T = 1 is the plain sigmoid of the logit; any T divides that same logit
+    np.testing.assert_allclose(special.logit(cT) * T, special.logit(c1), rtol=1e-9, atol=1e-9)
+    big = oracle_mod.confidence(h, anchor, x, W1, w, 1.0, np.full(gamma, 1e30, np.float32))["c"]
+    np.testing.assert_allclose(big, 0.5, atol=1e-12)
+
+
+def test_survival_is_cumulative_product_and_never_increases(oracle_mod):
+    B, gamma, d, r, V = 6, 12, 40, 16, 100
+    h, anchor, x, W1, w, T = _conf_inputs(B, gamma, d, r, V, 4)
+    out = oracle_mod.confidence(h, anchor, x, W1, w, 2.0, T)
+    c, P64, P32 = out["c"], out["P64"], out["P32"]
+    np.testing.assert_allclose(P64[:, 0], c[:, 0], rtol=1e-15)
+    np.testing.assert_allclose(P64[:, 1:] / P64[:, :-1], c[:, 1:], rtol=1e-12)
+    assert (np.diff(P64, axis=1) <= 0).all() and (P64 > 0).all() and (P64 <= 1).all()
+    assert (np.diff(P32.astype(np.float64), axis=1) <= 0).all()
+    np.testing.assert_allclose(P32, P64, rtol=1e-5)
+    # the fp32 product takes one rounding per step, with each factor rounded to fp32 first
+    np.testing.assert_array_equal(P32[:, 0], c[:, 0].astype(np.float32))
+
+
+def test_confidence_rejects_bad_temperature(oracle_mod):
+    h, anchor, x, W1, w, T = _conf_inputs(1, 2, 8, 4, 10, 5)
+    with pytest.raises(ValueError):
+        oracle_mod.confidence(h, anchor, x, W1, w, 0.0, np.array([1.0, 0.0], np.float32))
+
+
+# ---------------------------------------------------------------------------
+# Hardware-aware prefix scheduler (wispaper.ai "The Hardware-Aware Prefix
+# Scheduler"; gdymind.com "DSpark", section 6)
+# ---------------------------------------------------------------------------
+def _objective(P, L, Tstep):
+    """Expected tokens per second of a verify-length choice, exact numerator."""
+    B = P.shape[0]
+    num = B << 48
+    for b in range(B):
+        for k in range(L[b]):
+            num += math.floor(float(P[b, k]) * 2.0**48)
+    return math.ldexp(float(num) / float(Tstep[B + sum(L)]), -48)
+
+
+def _tables(B, gamma, rng):
+    n = B * (gamma + 1) + 1
+    yield np.full(n, 1000.0)                                          # flat
+    yield 1000.0 + 90.0 * np.arange(n)                                # linear
+    yield 500.0 + 300.0 * np.maximum(0, np.arange(n) - B - 2)         # knee
+    yield rng.uniform(100.0, 2000.0, n)                               # arbitrary
+    yield np.sort(rng.uniform(100.0, 2000.0, n))                      # increasing staircase
+
+
+@pytest.mark.parametrize("B,gamma", [(1, 1), (1, 4), (2, 3), (3, 2), (3, 4), (2, 4)])
+def test_schedule_matches_brute_force_enumeration(oracle_mod, B, gamma):
+    rng = np.random.default_rng(100 * B + gamma)
+    for trial in range(6):
+        P = synth.monotone_scores(B, gamma, seed=trial * 31 + B, tie_frac=0.3 if trial % 2 else 0.0,
+                                  zero_frac=0.3 if trial == 4 else 0.0)
+        for Tstep in _tables(B, gamma, rng):
+            L, N, F, _ = oracle_mod.schedule(P, Tstep)
+            best, best_n = -1.0, None
+            for Ls in itertools.product(range(gamma + 1), repeat=B):
+                f = _objective(P, Ls, Tstep)
+                if f > best:
+                    best, best_n = f, sum(Ls)
+                elif f == best:
+                    best_n = min(best_n, sum(Ls))
+            assert F == best
+            assert _objective(P, L, Tstep) == best
+            assert N == int(L.sum()) == best_n
+
+
+def test_schedule_flat_curve_verifies_everything(oracle_mod):
+    B, gamma = 4, 8
+    P = synth.monotone_scores(B, gamma, seed=9)
+    L, N, F, _ = oracle_mod.schedule(P, np.full(B * (gamma + 1) + 1, 20000.0))
+    assert (L == gamma).all() and N == B * gamma
+
+
+def test_schedule_steep_curve_verifies_nothing(oracle_mod):
+    B, gamma = 4, 8
+    P = synth.monotone_scores(B, gamma, seed=9)
+    n = np.arange(B * (gamma + 1) + 1, dtype=np.float64)
+    L, N, F, _ = oracle_mod.schedule(P, 1000.0 * 4.0 ** n)
+    assert (L == 0).all() and N == 0 and F == B / (1000.0 * 4.0 ** B)
+    assert F * 1e6 == pytest.approx(B / 256.0 * 1e3)   # tokens per second at a 256 ms step
+
+
+def test_schedule_lengths_are_prefixes_of_the_global_order(oracle_mod):
+    B, gamma = 16, 6
+    P = synth.monotone_scores(B, gamma, seed=4, tie_frac=0.4)
+    Tstep = 1000.0 + 40.0 * np.arange(B * (gamma + 1) + 1)
+    L, N, F, F_all = oracle_mod.schedule(P, Tstep)
+    assert 0 < N < B * gamma and F == F_all.max() and int(np.argmax(F_all)) == N
+    # every kept score is >= every dropped one
+    kept = np.concatenate([P[b, :L[b]] for b in range(B)])
+    dropped = np.concatenate([P[b, L[b]:] for b in range(B)])
+    assert kept.min() >= dropped.max()
+
+
+def test_schedule_worked_examples_of_the_pages(oracle_mod):
+    with open(os.path.join(GOLDEN, "scheduler_worked_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        P = np.array(case["P"], dtype=np.float32)
+        L, N, F, F_all = oracle_mod.schedule(P, np.array(case["tstep_us"]))
+        assert L.tolist() == case["expected_L"], case["name"]
+        np.testing.assert_allclose(F_all[:len(case["F_by_N"])], case["F_by_N"], rtol=2e-4)
+
+
+def test_schedule_rejects_scores_outside_unit_interval(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.schedule(np.array([[1.5, 0.5]], np.float32), np.ones(4))
+
+
+# ---------------------------------------------------------------------------
+# Strict prefix-match verification (seventnews.com article: the first rejected
+# token and everything after it are dropped)
+# ---------------------------------------------------------------------------
+def test_verify_special_cases(oracle_mod):
+    gamma = 5
+    x = np.array([[1, 2, 3, 4, 5]] * 5, np.int32)
+    t = np.array([[1, 2, 3, 4, 5, 6],      # all agree
+                  [9, 2, 3, 4, 5, 6],      # first disagrees
+                  [1, 2, 9, 4, 5, 6],      # third disagrees
+                  [1, 2, 3, 4, 9, 6],      # fifth disagrees, beyond L
+                  [1, 2, 3, 4, 5, 6]], np.int32)
+    L = np.array([5, 3, 4, 3, 0], np.int32)
+    acc, bonus = oracle_mod.verify(x, L, t)
+    assert acc.tolist() == [5, 0, 2, 3, 0]
+    assert bonus.tolist() == [6, 9, 9, 4, 1]
+
+
+def test_verify_random_against_mask_formulation(oracle_mod):
+    x, L, t = synth.verify_inputs(300, 9, 50, seed=2, agree=0.8)
+    acc, bonus = oracle_mod.verify(x, L, t)
+    k = np.arange(9)[None, :]
+    bad = (x != t[:, :9]) & (k < L[:, None])
+    expect = np.where(bad.any(axis=1), bad.argmax(axis=1), L)
+    np.testing.assert_array_equal(acc, expect)
+    np.testing.assert_array_equal(bonus, t[np.arange(300), expect])
+
+
+def test_verify_rejects_length_beyond_gamma(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.verify(np.zeros((1, 3), np.int32), np.array([4], np.int32),
+                          np.zeros((1, 4), np.int32))
