@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the DSpark drafter-head hot path on B200.
+
+One step = one draft block through the whole path: Markov-head drafting of gamma
+tokens for every request (dspark_draft_step), confidence + STS + survival product
+(dspark_confidence_sts), the prefix scheduler (dspark_schedule_prefix) and strict
+prefix-match verification (dspark_verify_prefix).  The metric is draft tokens per
+second, B * gamma / step time, summed over ranks.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload qwen3-8b]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+
+With N > 1 (torchrun, one process per GPU) every rank drafts its own B requests
+(weak scaling) and the survival scores of all ranks are all-gathered over NCCL
+before the scheduler, which then decides verify lengths over the global batch.
+
+Inputs are synthetic and seeded (synth.py).  U alone (311 MB at the default
+workload) is larger than L2, and L2 is also flushed between timed steps.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "draft tokens/s (Markov head+confidence+schedule+verify); % of HBM/TC roofline"
+UNIT = "tokens/s"
+DRAFT_SRC = os.path.join(ROOT, "speculative_decoding_drafter_head_b200", "csrc", "markov_draft.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "markov_draft_traffic.json")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def _kernel_sha():
+    with open(DRAFT_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _traffic_per_launch(workload_name):
+    """DRAM bytes per draft launch from the committed ncu summary, if the kernel is unchanged."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("kernel_sha") == _kernel_sha() and t.get("workload") == workload_name:
+            return float(t["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_step(wl, inp, bs, target_rows, oracle):
+    """The oracle's whole path on the listed requests (one bounded sample of a step)."""
+    bs = list(bs)
+    U = synth.u_requests(wl, bs) if inp.U is None else inp.U[bs]
+    h = synth.h_requests(wl, bs) if inp.h is None else inp.h[bs]
+    x, _, _ = oracle.draft(U, inp.anchor[bs], inp.W1, inp.W2, mode=wl.mode, tau=wl.tau,
+                           seed=wl.seed, b_index=np.array(bs, np.int32))
+    conf = oracle.confidence(h, inp.anchor[bs], x, inp.W1, inp.w, inp.b_conf, inp.T)
+    sub = wl.with_(B=len(bs))
+    L, _, _, _ = oracle.schedule(conf["P32"], synth.tstep_us(sub))
+    oracle.verify(x, L, target_rows)
+    return x
+
+
+def run_reference(args, wl):
+    """The CPU oracle as the reference arm: bounded samples of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    inp = synth.make_inputs(wl, with_u=False, with_h=False)
+    sample = list(range(min(wl.B, args.ref_sample)))
+    target = synth.targets(wl, np.zeros((len(sample), wl.gamma), np.int32), sample)
+    for _ in range(args.warmup):
+        cpu_oracle_step(wl, inp, sample, target, oracle)
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        cpu_oracle_step(wl, inp, sample, target, oracle)
+        t.append(time.perf_counter() - t0)
+    sec = sum(t)
+    value = len(sample) * wl.gamma * args.steps / sec
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "gamma": wl.gamma, "V": wl.V, "r": wl.r,
+                   "d": wl.d, "mode": "gumbel" if wl.mode else "greedy"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{len(sample)} of {wl.B} requests per step, whole path"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, inp, target, budget_s):
+    """Time the oracle on a growing sample of requests until about budget_s of CPU work."""
+    import oracle
+    oracle.build()
+    n = 1
+    spent = 0.0
+    while True:
+        bs = list(range(n))
+        t0 = time.perf_counter()
+        cpu_oracle_step(wl, inp, bs, target[:n], oracle)
+        dt = time.perf_counter() - t0
+        spent += dt
+        if dt >= budget_s / 3 or n >= wl.B or spent >= budget_s:
+            break
+        n = min(wl.B, max(n + 1, int(n * min(8.0, budget_s / 2 / max(dt, 1e-3)))))
+    return {"value": n * wl.gamma / dt, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{n} of {wl.B} requests, one full step "
+                                        f"(draft, confidence, schedule, verify), {dt:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3-8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--ref-sample", type=int, default=4)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import speculative_decoding_drafter_head_b200 as ds
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    B, gamma, V = wl.B, wl.gamma, wl.V
+    wlg = wl.with_(B=B * world)                 # the global batch across ranks
+    bs = range(rank * B, (rank + 1) * B)
+
+    # ---------------- inputs (host, seeded) and device copies
+    W1h, W2h = synth.w1(wl), synth.w2(wl)
+    Uh = synth.u_requests(wlg, bs)
+    hh = synth.h_requests(wlg, bs)
+    anchor_h = synth.anchors(wlg)[rank * B:(rank + 1) * B].copy()
+    wh, Th = synth.conf_w(wl), synth.temperatures(wl)
+    Tstep_h = synth.tstep_us(wlg)
+
+    def bf(a):
+        return torch.from_numpy(a).view(torch.bfloat16).cuda()
+
+    U, h, W1, W2, w = bf(Uh), bf(hh), bf(W1h), bf(W2h), bf(wh)
+    anchor = torch.from_numpy(anchor_h).cuda()
+    T = torch.from_numpy(Th).cuda()
+    Tstep = torch.from_numpy(Tstep_h).cuda()
+    ws = torch.empty(ds.workspace_bytes(B * world, gamma, V), dtype=torch.uint8, device="cuda")
+    x = torch.empty(B, gamma, dtype=torch.int32, device="cuda")
+    lx = torch.empty(B, gamma, dtype=torch.float32, device="cuda")
+    c = torch.empty(B, gamma, dtype=torch.float32, device="cuda")
+    P = torch.empty(B, gamma, dtype=torch.float32, device="cuda")
+    Pg = torch.empty(B * world, gamma, dtype=torch.float32, device="cuda")
+    Lg = torch.empty(B * world, dtype=torch.int32, device="cuda")
+    Nst = torch.empty(1, dtype=torch.int32, device="cuda")
+    obj = torch.empty(1, dtype=torch.float64, device="cuda")
+    acc = torch.empty(B, dtype=torch.int32, device="cuda")
+    bonus = torch.empty(B, dtype=torch.int32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    # target tokens: the target model agrees with the drafts w.p. q_k (from a first draft)
+    ds.draft_step(U, anchor, W1, W2, x, lx, ws, mode=wl.mode, temperature=wl.tau, seed=wl.seed,
+                  b_offset=rank * B)
+    torch.cuda.synchronize()
+    target_h = synth.targets(wlg, x.cpu().numpy(), bs)
+    target = torch.from_numpy(target_h).cuda()
+
+    ev_draft = []
+
+    def step(record=None):
+        e0 = e1 = None
+        if record is not None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        ds.draft_step(U, anchor, W1, W2, x, lx, ws, mode=wl.mode, temperature=wl.tau,
+                      seed=wl.seed, b_offset=rank * B)
+        if record is not None:
+            e1.record(stream)
+            record.append((e0, e1))
+        ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P)
+        if world > 1:
+            dist.all_gather_into_tensor(Pg, P)
+            ds.schedule_prefix(Pg, Tstep, Lg, Nst, obj, ws)
+            Lloc = Lg[rank * B:(rank + 1) * B]
+        else:
+            ds.schedule_prefix(P, Tstep, Lg, Nst, obj, ws)
+            Lloc = Lg
+        ds.verify_prefix(x, Lloc, target, acc, bonus)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ds.get_error() == 0, "device error during warm-up"
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ev = []
+    for _ in range(args.steps):
+        flush.zero_()                                   # evict L2 between timed steps
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step(ev_draft)
+        e1.record(stream)
+        step_ev.append((e0, e1))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    draft_ms = [a.elapsed_time(b) for a, b in ev_draft]
+    total_ms = sum(step_ms)
+    assert ds.get_error() == 0, "device error during the timed steps"
+
+    # ---------------- end to end through the public API with host buffers
+    pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+    U_pin, h_pin = pin(Uh).view(torch.bfloat16), pin(hh).view(torch.bfloat16)
+    anchor_pin, target_pin = pin(anchor_h), pin(target_h)
+    out_x = torch.empty(B, gamma, dtype=torch.int32).pin_memory()
+    out_L = torch.empty(B, dtype=torch.int32).pin_memory()
+    out_acc = torch.empty(B, dtype=torch.int32).pin_memory()
+    out_bonus = torch.empty(B, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (U_pin, h_pin, anchor_pin, target_pin))
+    d2h = sum(t.numel() * t.element_size() for t in (out_x, out_L, out_acc, out_bonus))
+
+    def e2e_step():
+        U.copy_(U_pin, non_blocking=True)
+        h.copy_(h_pin, non_blocking=True)
+        anchor.copy_(anchor_pin, non_blocking=True)
+        target.copy_(target_pin, non_blocking=True)
+        step()
+        out_x.copy_(x, non_blocking=True)
+        out_L.copy_(Lg[rank * B:(rank + 1) * B] if world > 1 else Lg, non_blocking=True)
+        out_acc.copy_(acc, non_blocking=True)
+        out_bonus.copy_(bonus, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ev = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e2e_step()
+        e1.record(stream)
+        e2e_ev.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    assert ds.get_error() == 0, "device error during the end-to-end steps"
+
+    # ---------------- max over ranks
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms, statistics.mean(draft_ms)], dtype=torch.float64,
+                         device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms, draft_mean = (float(v) for v in t.tolist())
+    else:
+        draft_mean = statistics.mean(draft_ms)
+
+    tokens = B * world * gamma * args.steps
+    value = tokens / (total_ms / 1e3)
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    if rank == 0:
+        hbm_gbs, tflops, peak_kind = _peaks()
+        algo_bytes = gamma * (wl.r * V * 2 + B * V * 2)          # W2 + U_k per position
+        achieved = algo_bytes / (draft_mean / 1e3) / 1e9
+        flops = gamma * 2.0 * B * wl.r * V
+        t_hbm = algo_bytes / (hbm_gbs * 1e9)
+        t_tc = flops / (tflops * 1e12)
+        roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "achieved": achieved,
+                "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
+                "traffic": _traffic_per_launch(wl.name), "kernel": "markov_draft_kernel",
+                "kernel_ms": draft_mean, "algorithmic_bytes": algo_bytes,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6650 GB/s"}
+        cpu = None
+        if world == 1:
+            inp = synth.Inputs(wl=wl, W1=W1h, W2=W2h, U=Uh, h=hh, anchor=anchor_h, w=wh, T=Th,
+                               Tstep=Tstep_h, b_conf=wl.b_conf)
+            cpu = cpu_baseline(wl, inp, target_h, args.cpu_budget)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B_per_gpu": B, "gamma": gamma, "V": V, "r": wl.r,
+                       "d": wl.d, "mode": "gumbel" if wl.mode else "greedy",
+                       "parallelism": f"dp{world}", "l2_flush": True},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk,
+            "draft_kernel_ms": {"mean": draft_mean, "min": min(draft_ms), "max": max(draft_ms)},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

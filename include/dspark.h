@@ -1,0 +1,171 @@
+/*
+ * dspark.h -- C ABI of the DSpark drafter-head hot path on one B200 (sm_100a).
+ *
+ * The method is described on three web pages about DSpark:
+ *   [G] gdymind.com, "DSpark: DeepSeek's new speculative decoding work (Video + Blog)"
+ *   [W] wispaper.ai, "DSpark: Overcoming the Efficiency Wall in LLM Speculative Decoding"
+ *   [S] seventnews.com, "DeepSeek's DSpark just fixed the two things that held back
+ *       faster AI inference"
+ *
+ * Conventions shared by every call:
+ *   - Every array argument is caller-owned DEVICE memory, contiguous and row-major.
+ *     The library never allocates or frees device memory and keeps no pointer
+ *     after a call returns.
+ *   - bf16 arrays are passed as `const void*` (2-byte bf16 storage).
+ *   - `stream` is the caller's cudaStream_t.  All work is enqueued on it and is
+ *     asynchronous; no call synchronises except dspark_get_error.
+ *   - The return value is a dspark_status.  Host-side argument checks run before
+ *     anything is enqueued; on a non-zero return nothing was enqueued.
+ *   - Problems seen on the device (an out-of-range token id, scores that are not
+ *     non-increasing, a wait that ran out) are recorded in a per-device error
+ *     word that dspark_get_error reads and clears.
+ *   - Not thread-safe across concurrent calls that share a workspace.
+ */
+#ifndef DSPARK_H
+#define DSPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dspark_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    DSPARK_OK = 0,
+    DSPARK_INVALID_ARG = 1,       /* null pointer, bad size, misaligned pointer   */
+    DSPARK_UNSUPPORTED_SHAPE = 2, /* a size outside what the kernels support     */
+    DSPARK_WORKSPACE_TOO_SMALL = 3,
+    DSPARK_NOT_MONOTONE = 4,      /* device: scores increase along a request      */
+    DSPARK_CUDA_ERROR = 5,        /* a CUDA runtime/driver call failed            */
+    DSPARK_TIMEOUT = 6,           /* device: a bounded wait ran out               */
+    DSPARK_INVALID_TOKEN = 7      /* device: a token id or length out of range    */
+} dspark_status;
+
+/* Text for a status code (static storage). */
+const char *dspark_status_string(int status);
+
+/* Number of bytes of device workspace dspark_draft_step and dspark_schedule_prefix
+ * need for these sizes (the larger of the two).  The workspace must be 256-byte
+ * aligned; its contents need no initialisation and are overwritten by each call. */
+size_t dspark_workspace_bytes(int B, int gamma, int V, int r);
+
+/*
+ * Markov-head drafting, all gamma positions of one draft block.
+ * [G] section 4 "Semi-Autoregressive Generation" (sequential stage, Markov head:
+ * first-order transition B = W1 W2 with W1 [V, r] an embedding table and W2 [r, V]
+ * a logits projection, r = 256) and section 4 "Parallel stage" (the anchor is the
+ * first prediction position, so gamma inputs give gamma logits).
+ *
+ * For k = 1..gamma, with x_0 = anchor[b]:
+ *   l_k(v) = U[b, k-1, v] + sum_j W1[x_{k-1}, j] W2[j, v]         (fp32 accumulate)
+ *   mode 0 (greedy):     x_k = argmax_v l_k(v), smallest v among equal maxima
+ *   mode 1 (Gumbel-max): x_k = argmax_v l_k(v) / temperature + g(b + b_offset, k, v)
+ *     with g = -ln(-ln u), u = ((w >> 9) + 0.5) 2^-23 and w word (v mod 4) of
+ *     Philox4x32-10(counter = (v / 4, k - 1, b + b_offset, 0),
+ *                   key = (low 32 bits of seed, high 32 bits of seed)).
+ *   x_out[b, k-1] = x_k;  logit_x_out[b, k-1] = l_k(x_k) (the unperturbed logit).
+ * The [B, V] logits are never written to memory.
+ *
+ *   U        [B, gamma, V] bf16   backbone base logits U_k
+ *   anchor   [B] int32            x_0; must lie in [0, V)
+ *   W1       [V, r] bf16          Markov embedding table
+ *   W2       [r, V] bf16          logits projection
+ *   x_out    [B, gamma] int32     drafted tokens
+ *   logit_x_out [B, gamma] fp32
+ *   workspace, workspace_bytes    >= dspark_workspace_bytes(B, gamma, V, r)
+ * Supported sizes: 1 <= B <= 1024, 1 <= gamma <= 64, r == 256, 64 <= V <= 2^24,
+ * V % 8 == 0; U, W1, W2 16-byte aligned.  temperature > 0 in mode 1.
+ * An anchor outside [0, V) records DSPARK_INVALID_TOKEN and is read as token 0.
+ * The kernel is a cooperative launch of one CTA per SM whose steps are joined
+ * by a grid barrier; every device-side wait is bounded (dspark_set_wait_timeout_ns)
+ * and records DSPARK_TIMEOUT instead of hanging.
+ */
+int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, const void *W2,
+                      int B, int gamma, int V, int r, int mode, float temperature,
+                      uint64_t seed, int b_offset, int32_t *x_out, float *logit_x_out,
+                      void *workspace, size_t workspace_bytes, dspark_stream_t stream);
+
+/*
+ * Confidence head with Sequential Temperature Scaling and prefix survival.
+ * [G] section 5 "Confidence-Scheduled Verification" (linear projection then
+ * sigmoid over the backbone hidden state at position k and the Markov embedding
+ * of the previous draft token; temperature scaling per position) and [S]
+ * ("per-position prefix survival probabilities", a cumulative product).
+ *
+ *   z_{b,k} = sum_i w[i] h[b, k-1, i] + sum_j w[d + j] W1[x_{k-1}, j] + b_conf
+ *   c_{b,k} = 1 / (1 + exp(-z_{b,k} / T[k-1]))
+ *   P_{b,k} = P_{b,k-1} * c_{b,k} in fp32, P_{b,0} = 1
+ * with x_0 = anchor[b], x_{k-1} = x[b, k-2] for k >= 2.
+ *
+ *   h [B, gamma, d] bf16;  anchor [B] int32;  x [B, gamma] int32 (last column unused)
+ *   W1 [V, r] bf16;  w [d + r] bf16;  T [gamma] fp32 (> 0)
+ *   c_out, P_out [B, gamma] fp32
+ * Supported sizes: 1 <= B, 1 <= gamma <= 64, d % 8 == 0, r % 8 == 0; h, W1, w
+ * 16-byte aligned.  A token id outside [0, V) records DSPARK_INVALID_TOKEN and is
+ * read as 0.
+ */
+int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x,
+                          const void *W1, const void *w, float b_conf, const float *T,
+                          int B, int gamma, int d, int r, int V, float *c_out, float *P_out,
+                          dspark_stream_t stream);
+
+/*
+ * Hardware-aware prefix scheduler: per-request verify lengths that maximise
+ * expected accepted tokens per unit time.
+ * [W] "The Hardware-Aware Prefix Scheduler" (throughput maximisation against a
+ * steps-per-second curve) and [G] section 6 ("global throughput maximization").
+ *
+ * Scores P[b, k-1] (non-increasing in k, within [0, 1]) are ordered by
+ * (P desc, b asc, k asc); q = floor(P 2^48); S_N = sum of the first N q's;
+ *   F(N) = double(B 2^48 + S_N) / Tstep_us[B + N],   N = 0 .. B gamma
+ * (int64 sum, round-to-nearest conversion and division).  N* = smallest N with
+ * the largest F; L_out[b] = number of request b's entries among the first N*.
+ *
+ *   P [B, gamma] fp32;  Tstep_us [B (gamma + 1) + 1] fp64, Tstep_us[n] > 0 is the
+ *   time of one target step that verifies n tokens (each request feeds its
+ *   anchor/bonus position plus L_b drafts, so n = B + sum L).
+ *   L_out [B] int32;  N_out [1] int32 (N*);  objective_out [1] fp64 = F(N*) 2^-48,
+ *   expected accepted tokens (bonus included) per unit of Tstep's time.
+ * Supported sizes: 1 <= B <= 32768, 1 <= gamma <= 64, B gamma <= 65536.
+ * A score outside [0, 1] or an increase along a request records
+ * DSPARK_NOT_MONOTONE (results are then unspecified but all writes stay in bounds).
+ */
+int dspark_schedule_prefix(const float *P, int B, int gamma, const double *Tstep_us,
+                           int32_t *L_out, int32_t *N_out, double *objective_out,
+                           void *workspace, size_t workspace_bytes, dspark_stream_t stream);
+
+/*
+ * Strict prefix-match verification.
+ * [S]: a block is verified in one target pass; the accepted tokens stick and the
+ * first rejected token and everything after it are dropped.
+ *   accepted_out[b] = smallest k-1 (1 <= k <= L[b]) with x[b, k-1] != target[b, k-1],
+ *                     or L[b] when the first L[b] drafts all agree
+ *   bonus_out[b]    = target[b, accepted_out[b]]
+ *   x [B, gamma] int32;  L [B] int32 in [0, gamma];  target [B, gamma + 1] int32
+ *   (the target model's tokens at positions 1..gamma+1).
+ * An L[b] outside [0, gamma] records DSPARK_INVALID_TOKEN and is clamped.
+ */
+int dspark_verify_prefix(const int32_t *x, const int32_t *L, const int32_t *target, int B,
+                         int gamma, int32_t *accepted_out, int32_t *bonus_out,
+                         dspark_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device into *status (DSPARK_OK when nothing was recorded). */
+int dspark_get_error(dspark_stream_t stream, int *status);
+
+/* Limit in nanoseconds for every device-side wait of dspark_draft_step
+ * (default 2e9).  Applies to launches made after the call. */
+int dspark_set_wait_timeout_ns(uint64_t ns);
+
+/* Test hook: the draft kernel's grid barrier waits for `extra` more arrivals than
+ * there are CTAs, so that its bounded wait runs out (0 restores normal use). */
+int dspark_debug_barrier_extra(int extra);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H */

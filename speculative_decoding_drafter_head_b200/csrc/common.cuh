@@ -1,0 +1,46 @@
+// common.cuh -- status codes, the per-device error word and small helpers.
+#pragma once
+#include <cstdint>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+// First problem seen on the device since the last dspark_get_error; 0 = none.
+__device__ unsigned int g_error_word;
+
+__device__ __forceinline__ void record_error(unsigned int code)
+{
+    atomicCAS(&g_error_word, 0u, code);
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// Monotone map of fp32 onto uint32 (larger float -> larger integer).
+__device__ __forceinline__ uint32_t float_order_bits(float f)
+{
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// 64-bit argmax key: larger value wins, then the smaller index.
+__device__ __forceinline__ unsigned long long argmax_key(float value, uint32_t index)
+{
+    return (static_cast<unsigned long long>(float_order_bits(value + 0.0f)) << 32) |
+           static_cast<unsigned long long>(0xFFFFFFFFu - index);
+}
+
+__device__ __forceinline__ uint32_t argmax_key_index(unsigned long long key)
+{
+    return 0xFFFFFFFFu - static_cast<uint32_t>(key);
+}
+
+}  // namespace dspark

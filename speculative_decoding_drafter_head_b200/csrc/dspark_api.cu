@@ -1,0 +1,324 @@
+// dspark_api.cu -- the C ABI (include/dspark.h): argument checks, TMA descriptors and
+// launches of the four hot-path kernels.  One translation unit holds every kernel so
+// that the per-device error word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "confidence_sts.cuh"
+#include "markov_draft.cuh"
+#include "ptx.cuh"
+#include "schedule_prefix.cuh"
+#include "verify_prefix.cuh"
+
+namespace {
+
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+std::atomic<int> g_barrier_extra{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    int major = 0;
+    bool draft_attr_set = false;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+int current_device(DeviceInfo **info)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return DSPARK_CUDA_ERROR;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (d.sms == 0) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            d.sms = 0;
+            return DSPARK_CUDA_ERROR;
+        }
+    }
+    if (d.major != 10) return DSPARK_UNSUPPORTED_SHAPE;   // built for sm_100a only
+    *info = &d;
+    return DSPARK_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// workspace layout shared by draft_step and schedule_prefix:
+//   [0, 256)          control words (counters, flags)
+//   [256, ...)        draft: argmax keys [gamma][B] u64
+//                     schedule: ranks [n] i32, then fixed-point scores [n] i64
+constexpr size_t kCtlBytes = 256;
+
+size_t draft_ws(int B, int gamma) { return kCtlBytes + static_cast<size_t>(B) * gamma * 8; }
+
+size_t sched_ws(int n)
+{
+    return kCtlBytes + round_up(static_cast<size_t>(n) * 4, 256) + static_cast<size_t>(n) * 8;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_CUDA_ERROR; }
+
+}  // namespace
+
+extern "C" {
+
+const char *dspark_status_string(int status)
+{
+    switch (status) {
+    case DSPARK_OK: return "ok";
+    case DSPARK_INVALID_ARG: return "invalid argument";
+    case DSPARK_UNSUPPORTED_SHAPE: return "unsupported shape or device";
+    case DSPARK_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DSPARK_NOT_MONOTONE: return "scores outside [0,1] or increasing along a request";
+    case DSPARK_CUDA_ERROR: return "CUDA error";
+    case DSPARK_TIMEOUT: return "device wait timed out";
+    case DSPARK_INVALID_TOKEN: return "token id or verify length out of range";
+    default: return "unknown status";
+    }
+}
+
+size_t dspark_workspace_bytes(int B, int gamma, int V, int r)
+{
+    (void)V;
+    (void)r;
+    if (B < 1 || gamma < 1) return 0;
+    const size_t a = draft_ws(B, gamma);
+    const size_t b = sched_ws(B * gamma);
+    return a > b ? a : b;
+}
+
+int dspark_set_wait_timeout_ns(uint64_t ns)
+{
+    if (ns == 0) return DSPARK_INVALID_ARG;
+    g_timeout_ns.store(ns);
+    return DSPARK_OK;
+}
+
+int dspark_debug_barrier_extra(int extra)
+{
+    if (extra < 0) return DSPARK_INVALID_ARG;
+    g_barrier_extra.store(extra);
+    return DSPARK_OK;
+}
+
+int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, const void *W2, int B,
+                      int gamma, int V, int r, int mode, float temperature, uint64_t seed,
+                      int b_offset, int32_t *x_out, float *logit_x_out, void *workspace,
+                      size_t workspace_bytes, dspark_stream_t stream)
+{
+    namespace D = dspark::draft;
+    if (!U || !anchor || !W1 || !W2 || !x_out || !logit_x_out || !workspace)
+        return DSPARK_INVALID_ARG;
+    if (!aligned(U, 16) || !aligned(W1, 16) || !aligned(W2, 16) || !aligned(anchor, 4) ||
+        !aligned(x_out, 4) || !aligned(logit_x_out, 4) || !aligned(workspace, 256))
+        return DSPARK_INVALID_ARG;
+    if (mode != 0 && mode != 1) return DSPARK_INVALID_ARG;
+    if (mode == 1 && !(temperature > 0.0f)) return DSPARK_INVALID_ARG;
+    if (b_offset < 0) return DSPARK_INVALID_ARG;
+    if (B < 1 || B > D::kMaxB || gamma < 1 || gamma > 64 || r != D::kRank || V < 64 ||
+        V > (1 << 24) || V % 8 != 0)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < draft_ws(B, gamma)) return DSPARK_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    if (int st = current_device(&dev)) return st;
+    EncodeTiledFn encode = encode_tiled();
+    if (!encode) return DSPARK_CUDA_ERROR;
+
+    const int ub = B < D::kMTile ? B : D::kMTile;
+    CUtensorMap tm_w2, tm_u;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(V), static_cast<cuuint64_t>(r)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(V) * 2};
+        const cuuint32_t box[2] = {D::kTileN, static_cast<cuuint32_t>(r)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (encode(&tm_w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(W2), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return DSPARK_CUDA_ERROR;
+    }
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(V), static_cast<cuuint64_t>(gamma),
+                                    static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(V) * 2,
+                                       static_cast<cuuint64_t>(V) * 2 * gamma};
+        const cuuint32_t box[3] = {D::kTileN, 1, static_cast<cuuint32_t>(ub)};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (encode(&tm_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(U), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return DSPARK_CUDA_ERROR;
+    }
+
+    if (!dev->draft_attr_set) {
+        if (cudaFuncSetAttribute(D::markov_draft_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 D::kDynSmem) != cudaSuccess)
+            return DSPARK_CUDA_ERROR;
+        dev->draft_attr_set = true;
+    }
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    D::Params prm;
+    prm.anchor = anchor;
+    prm.W1 = static_cast<const uint16_t *>(W1);
+    prm.B = B;
+    prm.gamma = gamma;
+    prm.V = V;
+    prm.mode = mode;
+    prm.inv_tau = mode == 1 ? 1.0f / temperature : 1.0f;
+    prm.seed_lo = static_cast<uint32_t>(seed);
+    prm.seed_hi = static_cast<uint32_t>(seed >> 32);
+    prm.b_offset = b_offset;
+    prm.x_out = x_out;
+    prm.logit_out = logit_x_out;
+    prm.barrier = reinterpret_cast<unsigned int *>(ws);
+    prm.abort_flag = reinterpret_cast<unsigned int *>(ws + 4);
+    prm.slots = reinterpret_cast<unsigned long long *>(ws + kCtlBytes);
+    prm.ntiles_total = (V + D::kTileN - 1) / D::kTileN;
+    prm.ub = ub;
+    prm.timeout_ns = g_timeout_ns.load();
+    prm.barrier_extra = g_barrier_extra.load();
+
+    if (cudaMemsetAsync(ws, 0, draft_ws(B, gamma), stream) != cudaSuccess) return DSPARK_CUDA_ERROR;
+
+    const int grid = prm.ntiles_total < dev->sms ? prm.ntiles_total : dev->sms;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(D::kThreads);
+    cfg.dynamicSmemBytes = D::kDynSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel, tm_w2, tm_u, prm));
+}
+
+int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x, const void *W1,
+                          const void *w, float b_conf, const float *T, int B, int gamma, int d,
+                          int r, int V, float *c_out, float *P_out, dspark_stream_t stream)
+{
+    namespace C = dspark::conf;
+    if (!h || !anchor || !x || !W1 || !w || !T || !c_out || !P_out) return DSPARK_INVALID_ARG;
+    if (!aligned(h, 16) || !aligned(W1, 16) || !aligned(w, 16) || !aligned(anchor, 4) ||
+        !aligned(x, 4) || !aligned(T, 4) || !aligned(c_out, 4) || !aligned(P_out, 4))
+        return DSPARK_INVALID_ARG;
+    if (B < 1 || gamma < 1 || gamma > C::kMaxGamma || d < 8 || d % 8 != 0 || r < 8 ||
+        r % 8 != 0 || V < 1 || (d + r) * 2 > 200 * 1024)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    DeviceInfo *dev = nullptr;
+    if (int st = current_device(&dev)) return st;
+    const int smem = (d + r) * 2;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(C::confidence_sts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+        return DSPARK_CUDA_ERROR;
+    C::confidence_sts_kernel<<<B, C::kThreads, smem, stream>>>(
+        static_cast<const uint16_t *>(h), anchor, x, static_cast<const uint16_t *>(W1),
+        static_cast<const uint16_t *>(w), b_conf, T, B, gamma, d, r, V, c_out, P_out);
+    return from_cuda(cudaGetLastError());
+}
+
+int dspark_schedule_prefix(const float *P, int B, int gamma, const double *Tstep_us,
+                           int32_t *L_out, int32_t *N_out, double *objective_out, void *workspace,
+                           size_t workspace_bytes, dspark_stream_t stream)
+{
+    namespace S = dspark::sched;
+    if (!P || !Tstep_us || !L_out || !N_out || !objective_out || !workspace)
+        return DSPARK_INVALID_ARG;
+    if (!aligned(P, 4) || !aligned(Tstep_us, 8) || !aligned(L_out, 4) || !aligned(N_out, 4) ||
+        !aligned(objective_out, 8) || !aligned(workspace, 256))
+        return DSPARK_INVALID_ARG;
+    if (B < 1 || B > 32768 || gamma < 1 || gamma > 64 || static_cast<long long>(B) * gamma > 65536)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    const int n = B * gamma;
+    if (workspace_bytes < sched_ws(n)) return DSPARK_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    if (int st = current_device(&dev)) return st;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    S::Params prm;
+    prm.P = P;
+    prm.B = B;
+    prm.gamma = gamma;
+    prm.n = n;
+    prm.Tstep = Tstep_us;
+    prm.L_out = L_out;
+    prm.N_out = N_out;
+    prm.objective_out = objective_out;
+    prm.done = reinterpret_cast<unsigned int *>(ws);
+    prm.rank = reinterpret_cast<int32_t *>(ws + kCtlBytes);
+    prm.q_sorted = reinterpret_cast<long long *>(ws + kCtlBytes + round_up(static_cast<size_t>(n) * 4, 256));
+    if (cudaMemsetAsync(ws, 0, kCtlBytes, stream) != cudaSuccess) return DSPARK_CUDA_ERROR;
+    int grid = (n + S::kWarps - 1) / S::kWarps;
+    if (grid > 2 * dev->sms) grid = 2 * dev->sms;
+    S::schedule_prefix_kernel<<<grid, S::kThreads, 0, stream>>>(prm);
+    return from_cuda(cudaGetLastError());
+}
+
+int dspark_verify_prefix(const int32_t *x, const int32_t *L, const int32_t *target, int B,
+                         int gamma, int32_t *accepted_out, int32_t *bonus_out,
+                         dspark_stream_t stream)
+{
+    namespace Vf = dspark::verify;
+    if (!x || !L || !target || !accepted_out || !bonus_out) return DSPARK_INVALID_ARG;
+    if (!aligned(x, 4) || !aligned(L, 4) || !aligned(target, 4) || !aligned(accepted_out, 4) ||
+        !aligned(bonus_out, 4))
+        return DSPARK_INVALID_ARG;
+    if (B < 1 || gamma < 1 || gamma > 4096) return DSPARK_UNSUPPORTED_SHAPE;
+    DeviceInfo *dev = nullptr;
+    if (int st = current_device(&dev)) return st;
+    Vf::verify_prefix_kernel<<<(B + Vf::kThreads - 1) / Vf::kThreads, Vf::kThreads, 0, stream>>>(
+        x, L, target, B, gamma, accepted_out, bonus_out);
+    return from_cuda(cudaGetLastError());
+}
+
+int dspark_get_error(dspark_stream_t stream, int *status)
+{
+    if (!status) return DSPARK_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return DSPARK_CUDA_ERROR;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, dspark::g_error_word, sizeof v) != cudaSuccess)
+        return DSPARK_CUDA_ERROR;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(dspark::g_error_word, &zero, sizeof zero) != cudaSuccess)
+        return DSPARK_CUDA_ERROR;
+    *status = static_cast<int>(v);
+    return DSPARK_OK;
+}
+
+}  // extern "C"

@@ -23,8 +23,8 @@ from __future__ import annotations
 import math
 import os
 from concurrent.futures import ThreadPoolExecutor
-from dataclasses import dataclass, field, replace
-from typing import Callable, Optional, Sequence
+from dataclasses import dataclass, replace
+from typing import Optional, Sequence
 
 import numpy as np
 
@@ -221,6 +221,26 @@ def u_requests(wl: Workload, bs: Sequence[int]) -> np.ndarray:
 def u_all(wl: Workload) -> np.ndarray:
     """Base logits U [B, gamma, V] (bf16 bits)."""
     return u_requests(wl, range(wl.B))
+
+
+def u_all_device_zipf(wl: Workload, device: str = "cuda"):
+    """Zipf base logits U [B, gamma, V] built directly in device memory (torch bf16).
+
+    Same bytes as ``u_all``: the bf16 value table is made on the host and the
+    per-position rank permutation is pure integer arithmetic, done request by
+    request on the device to avoid a host copy of a multi-GB tensor.
+    """
+    import torch
+    assert wl.logits == "zipf"
+    table = torch.from_numpy(_zipf_table(wl).view(np.int16)).to(device)
+    out = torch.empty((wl.B, wl.gamma, wl.V), dtype=torch.int16, device=device)
+    v = torch.arange(wl.V, dtype=torch.int64, device=device)
+    for b in range(wl.B):
+        a, c = zipf_params(wl, b)
+        at = torch.from_numpy(a).to(device)
+        ct = torch.from_numpy(c).to(device)
+        out[b] = table[(at[:, None] * v[None, :] + ct[:, None]) % wl.V]
+    return out.view(torch.bfloat16)
 
 
 def h_requests(wl: Workload, bs: Sequence[int]) -> np.ndarray:
