@@ -155,15 +155,16 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     EncodeTiledFn encode = encode_tiled();
     if (!encode) return DSPARK_CUDA_ERROR;
 
-    const int ub = B < D::kMTile ? B : D::kMTile;
+    const int M = B <= 64 ? 64 : 128;
+    const int ub = B < M ? B : M;
     CUtensorMap tm_w2, tm_u;
     {
         const cuuint64_t dims[2] = {static_cast<cuuint64_t>(V), static_cast<cuuint64_t>(r)};
         const cuuint64_t strides[1] = {static_cast<cuuint64_t>(V) * 2};
-        const cuuint32_t box[2] = {D::kTileN, static_cast<cuuint32_t>(r)};
+        const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(D::kKSlice)};
         const cuuint32_t estr[2] = {1, 1};
         if (encode(&tm_w2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(W2), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return DSPARK_CUDA_ERROR;
@@ -173,7 +174,7 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
                                     static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(V) * 2,
                                        static_cast<cuuint64_t>(V) * 2 * gamma};
-        const cuuint32_t box[3] = {D::kTileN, 1, static_cast<cuuint32_t>(ub)};
+        const cuuint32_t box[3] = {D::kUnit, 1, static_cast<cuuint32_t>(ub)};
         const cuuint32_t estr[3] = {1, 1, 1};
         if (encode(&tm_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(U), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -207,14 +208,19 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     prm.barrier = reinterpret_cast<unsigned int *>(ws);
     prm.abort_flag = reinterpret_cast<unsigned int *>(ws + 4);
     prm.slots = reinterpret_cast<unsigned long long *>(ws + kCtlBytes);
-    prm.ntiles_total = (V + D::kTileN - 1) / D::kTileN;
+    prm.units_total = (V + D::kUnit - 1) / D::kUnit;
+    prm.M = M;
+    prm.w2_stages = M == 64 ? 4 : 3;
     prm.ub = ub;
+    prm.u_slot_bytes = M * D::kUnit * 2;   // a full M-row tile: the MMA reads all M rows
+    prm.u_slots = D::kURingBytes / prm.u_slot_bytes;
+    if (prm.u_slots > D::kUMaxSlots) prm.u_slots = D::kUMaxSlots;
     prm.timeout_ns = g_timeout_ns.load();
     prm.barrier_extra = g_barrier_extra.load();
 
     if (cudaMemsetAsync(ws, 0, draft_ws(B, gamma), stream) != cudaSuccess) return DSPARK_CUDA_ERROR;
 
-    const int grid = prm.ntiles_total < dev->sms ? prm.ntiles_total : dev->sms;
+    const int grid = prm.units_total < dev->sms ? prm.units_total : dev->sms;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3(grid);

@@ -6,18 +6,28 @@
 // U_k and picks x_k from them.
 //
 // One persistent cooperative kernel runs all gamma positions.  Each CTA owns a
-// contiguous slice of the vocabulary, cut into tiles of 32 columns, and for every
-// position k and every block of 128 requests it computes
+// contiguous slice of the vocabulary (a whole number of 32-column units, balanced
+// over the grid) cut into tiles of up to 256 columns, and for every position k and
+// every block of M requests it computes
 //     D[b, v] = sum_j A[b, j] W2[j, v],   A[b, :] = W1[x_{k-1, b}, :]
-// as M=128, N=32, K=256 tcgen05.mma (bf16 in, fp32 accumulate in TMEM).  The
-// epilogue adds U_k, applies greedy or Gumbel-max selection and keeps a running
+// as tcgen05.mma M=64/128, N<=256, K=16 (bf16 in, fp32 accumulate in TMEM), with W2
+// streamed by TMA in four K-slices of 64 rows (MN-major, 128-byte swizzle).  U_k is
+// added on the tensor core as well: each 32-column U tile, as staged by TMA (K-major,
+// 64-byte swizzle), is multiplied by a 32 x 32 identity into the same accumulator,
+// which is exact (bf16 times 1 into fp32).  The epilogue therefore reads finished
+// logits from TMEM, applies greedy or Gumbel-max selection and keeps a running
 // (max, index) per request row, so the [B, V] logits never reach memory.  Rows are
-// combined across CTAs by a 64-bit atomicMax on (ordered value, inverted index);
-// a bounded grid barrier ends each position, after which every CTA reads x_k for
-// the next gather and the CTA that owns the winning column writes the outputs.
+// combined across CTAs by a 64-bit atomicMax on (ordered value, inverted index); a
+// bounded grid barrier ends each position, after which every CTA reads x_k for the
+// next gather and the CTA that owns the winning column writes the outputs.
 //
-// Warp roles (192 threads): warps 0-3 epilogue (TMEM lanes 0-127) and A gather,
-// warp 4 TMA producer (W2 tile + U tile per stage), warp 5 MMA issuer + TMEM owner.
+// W2 is read with an L2 evict-last policy and U with evict-first: within one launch
+// W2 (at most 134 MB) is re-read every position and mostly stays in L2.
+//
+// Warp roles (352 threads): warps 0-7 epilogue and A gather (warps q and q + 4 read
+// TMEM lane quadrant q and split each tile's 32-column chunks between them), warp 8
+// W2 producer, warp 9 U producer, warp 10 MMA issuer and TMEM owner.  With B <= 64 the
+// MMA uses M = 64 (rows 16q..16q+15 sit in TMEM lanes 32q..32q+15), else M = 128.
 #pragma once
 #include <cuda.h>
 
@@ -27,22 +37,28 @@
 namespace dspark {
 namespace draft {
 
-constexpr int kTileN = 32;                       // vocabulary columns per tile
-constexpr int kRank = 256;                       // r, the contraction length
-constexpr int kMTile = 128;                      // requests per M tile
-constexpr int kStages = 6;                       // W2/U smem ring depth
-constexpr int kAcc = 4;                          // TMEM accumulator buffers
-constexpr int kABytes = kMTile * kRank * 2;      // 64 KB gathered W1 rows
-constexpr int kAChunk = kMTile * 128;            // one 64-column (128 B) K chunk
-constexpr int kW2Bytes = kTileN * kRank * 2;     // 16 KB per W2 tile
-constexpr int kUBytes = kMTile * kTileN * 2;     // 8 KB per U tile (max rows)
-constexpr int kStageBytes = kW2Bytes + kUBytes;  // 24 KB
-constexpr int kDynSmem = kABytes + kStages * kStageBytes + 1024;  // + alignment slack
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
-constexpr uint32_t kTmemCols = kAcc * kTileN;    // 128 columns
+constexpr int kUnit = 32;                         // columns per U box and epilogue chunk
+constexpr int kMaxUnits = 8;                      // 256 columns per MMA tile
+constexpr int kRank = 256;                        // r, the contraction length
+constexpr int kKSlice = 64;                       // W2 rows per ring stage
+constexpr int kKSlices = kRank / kKSlice;         // 4
+constexpr int kMaxW2Stages = 4;
+constexpr int kW2BoxBytes = 64 * kKSlice * 2;     // one TMA box: 64 columns x 64 rows
+constexpr int kW2StageBytes = 4 * kW2BoxBytes;    // 32 KB: 256 columns x 64 rows
+constexpr int kURingBytes = 62 * 1024;            // U tiles, M rows x 32 columns each
+constexpr int kUMaxSlots = 16;
+constexpr int kIdentBytes = 2 * 1024;             // 32 x 32 bf16 identity (B operand)
+constexpr int kAcc = 2;                           // TMEM accumulators of 256 columns
+constexpr uint32_t kTmemCols = 512;
+// A (M x 256 bf16) + W2 ring + U ring + identity: M = 64 with 4 W2 stages or M = 128 with 3
+constexpr int kDynSmem = 224 * 1024 + 1024;       // + alignment slack
+constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
+constexpr int kThreads = (kEpiWarps + 3) * 32;    // + W2 producer, U producer, MMA issuer
+constexpr int kWarpW2 = kEpiWarps, kWarpU = kEpiWarps + 1, kWarpMma = kEpiWarps + 2;
 constexpr int kMaxB = 1024;
-constexpr float kGumbelMax = 17.0f;              // above any noise value the epilogue makes
+constexpr int kMaxMTiles = kMaxB / 64;
+constexpr float kGumbelMax = 17.0f;               // above any noise value the epilogue makes
+constexpr uint32_t kWaitHintNs = 20000;           // longest hardware suspension per try_wait
 
 struct Params {
     const int32_t *anchor;
@@ -56,21 +72,48 @@ struct Params {
     unsigned long long *slots;   // [gamma][B] argmax keys, zeroed before launch
     unsigned int *barrier;       // grid barrier arrival counter, zeroed before launch
     unsigned int *abort_flag;    // set by any CTA that gives up, zeroed before launch
-    int ntiles_total;            // ceil(V / 32)
-    int ub;                      // rows of the U TMA box: min(B, 128)
+    int units_total;             // ceil(V / 32)
+    int M;                       // requests per MMA tile: 64 (B <= 64) or 128
+    int w2_stages;               // W2 ring depth (4 when M = 64, else 3)
+    int ub;                      // rows of the U TMA box: min(B, M)
+    int u_slots;                 // U ring depth
+    int u_slot_bytes;
     unsigned long long timeout_ns;
     int barrier_extra;
 };
 
 struct Ctl {
-    unsigned long long full[kStages];
-    unsigned long long empty[kStages];
+    unsigned long long w2_full[kMaxW2Stages];
+    unsigned long long w2_empty[kMaxW2Stages];
+    unsigned long long u_full[kUMaxSlots];
+    unsigned long long u_empty[kUMaxSlots];
     unsigned long long tfull[kAcc];
     unsigned long long tempty[kAcc];
     unsigned long long afull, aempty, drain;
     uint32_t tmem_base;
     int abort;
 };
+
+// A ring position: slot index and the parity of its current use.
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n)
+    {
+        if (++slot == n) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+// The t-th tile of a CTA that owns n_units units split into ntiles balanced tiles.
+__device__ __forceinline__ void tile_span(int t, int n_units, int ntiles, int &first, int &count)
+{
+    const int base = n_units / ntiles, extra = n_units % ntiles;
+    first = t * base + min(t, extra);
+    count = base + (t < extra ? 1 : 0);
+}
 
 __device__ __forceinline__ void give_up(Ctl &ctl, const Params &p, unsigned code)
 {
@@ -85,14 +128,12 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl &c
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 63u) == 0) {
-            if (*reinterpret_cast<volatile int *>(&ctl.abort)) return false;
-            if (globaltimer_ns() - t0 > p.timeout_ns) {
-                give_up(ctl, p, DSPARK_TIMEOUT);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
+        if (*reinterpret_cast<volatile int *>(&ctl.abort)) return false;
+        if (globaltimer_ns() - t0 > p.timeout_ns) {
+            give_up(ctl, p, DSPARK_TIMEOUT);
+            return false;
         }
     }
 }
@@ -101,7 +142,7 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, Ctl &c
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const Params &p)
 {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, kWaitHintNs)) {
         if (globaltimer_ns() - t0 > p.timeout_ns) {
             record_error(DSPARK_TIMEOUT);
             return;
@@ -109,14 +150,16 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const 
     }
 }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-
-__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int *ptr)
+// Wait for the last use of every slot of a ring of n slots after `issued` uses in total.
+__device__ __forceinline__ void drain_ring(uint32_t bar0, int n, long long issued, const Params &p)
 {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
+    for (int s = 0; s < n; ++s) {
+        const long long uses = issued / n + (s < issued % n ? 1 : 0);
+        if (uses > 0) wait_drain(bar0 + 8 * s, static_cast<uint32_t>((uses - 1) & 1), p);
+    }
 }
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // Philox4x32-10 (Salmon et al., SC'11): 10 rounds of the 4-word S-box with round
 // multipliers 0xD2511F53, 0xCD9E8D57 and key increments 0x9E3779B9, 0xBB67AE85.
@@ -148,38 +191,101 @@ __device__ __forceinline__ float gumbel_from_word(uint32_t w)
     return -__logf(e);
 }
 
-__device__ __forceinline__ void lds128(uint32_t addr, uint32_t &a, uint32_t &b, uint32_t &c,
-                                       uint32_t &d)
+__device__ __forceinline__ void sts128_zero(uint32_t addr)
 {
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
-                 : "r"(addr));
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, int4 v)
+__device__ __forceinline__ int checked_token(int tok, int V)
 {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
-// Token x_{k-1} of request b (k is 1-based): the anchor at k = 1, else the winner of
-// position k-1 read from the combined argmax keys.  Out-of-range ids are recorded and
-// replaced by 0 so that no gather leaves W1.
-__device__ __forceinline__ int prev_token(const Params &p, int b, int k)
-{
-    int tok;
-    if (k == 1) {
-        tok = p.anchor[b];
-    } else {
-        const unsigned long long key = __ldcg(&p.slots[static_cast<size_t>(k - 2) * p.B + b]);
-        tok = static_cast<int>(argmax_key_index(key));
-    }
-    if (tok < 0 || tok >= p.V) {
+    if (tok < 0 || tok >= V) {
         record_error(DSPARK_INVALID_TOKEN);
-        tok = 0;
+        return 0;
     }
     return tok;
+}
+
+// Running best of one request row over one 32-column chunk: l = acc + U, greedy or
+// Gumbel-max score s, strict improvement keeps the smallest column on ties.
+struct RowBest {
+    float s = -INFINITY;
+    float l = 0.0f;
+    uint32_t v = 0xFFFFFFFFu;
+};
+
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Largest of 32 values with three-input max (17 instructions instead of 31).
+__device__ __forceinline__ float max32(const float (&s)[32])
+{
+    float m[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) m[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+    m[10] = fmaxf(s[30], s[31]);
+    const float a = fmax3(m[0], m[1], m[2]), b = fmax3(m[3], m[4], m[5]);
+    const float c = fmax3(m[6], m[7], m[8]), d = fmaxf(m[9], m[10]);
+    return fmaxf(fmax3(a, b, c), d);
+}
+
+// Running best of one request row over one 32-column chunk of finished logits l
+// (U_k + bias, from TMEM): greedy or Gumbel-max score s; a strict improvement keeps
+// the smallest column on ties.
+__device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[32], int v0,
+                                             const Params &p, int k, int b_glob)
+{
+    float l[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) l[i] = __uint_as_float(a[i]);
+    if (v0 + kUnit > p.V) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (v0 + i >= p.V) l[i] = -INFINITY;
+    }
+    float s[32];
+    if (p.mode == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] = l[i];
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float lmax =
+                fmaxf(fmaxf(l[4 * q], l[4 * q + 1]), fmaxf(l[4 * q + 2], l[4 * q + 3]));
+            // exact pruning: noise cannot lift this group above the running best
+            const bool skip = !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best.s);
+            if (__all_sync(0xFFFFFFFFu, skip)) {
+                s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
+            } else {
+                const uint4 w = philox(make_uint4(static_cast<uint32_t>(v0 / 4 + q),
+                                                  static_cast<uint32_t>(k - 1),
+                                                  static_cast<uint32_t>(b_glob), 0u),
+                                       p.seed_lo, p.seed_hi);
+                s[4 * q + 0] = fmaf(l[4 * q + 0], p.inv_tau, gumbel_from_word(w.x));
+                s[4 * q + 1] = fmaf(l[4 * q + 1], p.inv_tau, gumbel_from_word(w.y));
+                s[4 * q + 2] = fmaf(l[4 * q + 2], p.inv_tau, gumbel_from_word(w.z));
+                s[4 * q + 3] = fmaf(l[4 * q + 3], p.inv_tau, gumbel_from_word(w.w));
+                if (skip) s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
+            }
+        }
+    }
+    const float mx = max32(s);
+    if (mx > best.s) {
+        int idx = 31;
+#pragma unroll
+        for (int i = 31; i >= 0; --i)
+            if (s[i] == mx) idx = i;
+        float li = l[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i)
+            if (i == idx) li = l[i];
+        best.s = mx;
+        best.l = li;
+        best.v = static_cast<uint32_t>(v0 + idx);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -188,24 +294,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t dyn_smem[];
     __shared__ Ctl ctl;
-    __shared__ unsigned long long row_key[kMaxB];
-    __shared__ float row_logit[kMaxB];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int M = p.M;
+    const int a_chunk = M * 128;                  // one 64-column K chunk of A
     const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     const uint32_t sA = base;
-    const uint32_t sStage = base + kABytes;
+    const uint32_t sW2 = base + static_cast<uint32_t>(M * kRank * 2);
+    const uint32_t sU = sW2 + static_cast<uint32_t>(p.w2_stages * kW2StageBytes);
+    const uint32_t sI = sU + kURingBytes;
 
     const int G = gridDim.x;
-    const int t_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.ntiles_total / G);
-    const int t_end =
-        static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.ntiles_total / G);
-    const int ntiles = t_end - t_begin;
-    const int num_mt = (p.B + kMTile - 1) / kMTile;
+    const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.units_total / G);
+    const int u_end =
+        static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.units_total / G);
+    const int n_units = u_end - u_begin;
+    const int ntiles = (n_units + kMaxUnits - 1) / kMaxUnits;
+    const int num_mt = (p.B + M - 1) / M;
 
-    const uint32_t bar_full = smem_u32(&ctl.full[0]);
-    const uint32_t bar_empty = smem_u32(&ctl.empty[0]);
+    const uint32_t bar_w2_full = smem_u32(&ctl.w2_full[0]);
+    const uint32_t bar_w2_empty = smem_u32(&ctl.w2_empty[0]);
+    const uint32_t bar_u_full = smem_u32(&ctl.u_full[0]);
+    const uint32_t bar_u_empty = smem_u32(&ctl.u_empty[0]);
     const uint32_t bar_tfull = smem_u32(&ctl.tfull[0]);
     const uint32_t bar_tempty = smem_u32(&ctl.tempty[0]);
     const uint32_t bar_afull = smem_u32(&ctl.afull);
@@ -213,25 +324,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_drain = smem_u32(&ctl.drain);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1 + 4);
+        for (int s = 0; s < p.w2_stages; ++s) {
+            mbar_init(bar_w2_full + 8 * s, 1);
+            mbar_init(bar_w2_empty + 8 * s, 1);
+        }
+        for (int s = 0; s < p.u_slots; ++s) {
+            mbar_init(bar_u_full + 8 * s, 1);
+            mbar_init(bar_u_empty + 8 * s, 1);
         }
         for (int a = 0; a < kAcc; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
-            mbar_init(bar_tempty + 8 * a, 4);
+            mbar_init(bar_tempty + 8 * a, kEpiWarps);
         }
-        mbar_init(bar_afull, 4);
+        mbar_init(bar_afull, kEpiWarps);
         mbar_init(bar_aempty, 1);
         mbar_init(bar_drain, 1);
         ctl.abort = 0;
         mbar_fence_init();
     }
-    if (warp == 5) {
+    if (threadIdx.x < 128) {
+        // 32 x 32 identity as an MN-major, 64-byte-swizzled B operand: row k holds 1.0
+        // at column k; 16-byte unit j of row k sits at unit j ^ ((k >> 1) & 3).
+        const int kr = threadIdx.x >> 2, j = threadIdx.x & 3;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (j == (kr >> 3)) {
+            const int e = kr & 7;                         // element within the unit
+            w[e >> 1] = (e & 1) ? 0x3F800000u : 0x00003F80u;
+        }
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                         sI + kr * 64 + ((j ^ ((kr >> 1) & 3)) << 4)),
+                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                     : "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == kWarpMma) {
         tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kWarpW2 && lane == 0) {
         tma_prefetch_desc(&tm_w2);
         tma_prefetch_desc(&tm_u);
     }
@@ -240,51 +370,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ TMA producer
+    if (warp == kWarpW2) {
+        // ------------------------------------------------------------ W2 producer
         if (lane == 0) {
             const uint64_t pol_w2 = l2_policy_evict_last();
-            const uint64_t pol_u = l2_policy_evict_first();
-            const uint32_t tx = kW2Bytes + static_cast<uint32_t>(p.ub) * kTileN * 2;
-            int stage = 0;
-            uint32_t phase = 0;
+            Ring w2;
             long long issued = 0;
             bool ok = true;
             for (int k = 1; k <= p.gamma && ok; ++k) {
                 for (int mt = 0; mt < num_mt && ok; ++mt) {
-                    for (int j = 0; j < ntiles; ++j) {
-                        if (!wait_phase(bar_empty + 8 * stage, phase ^ 1u, ctl, p)) {
-                            ok = false;
-                            break;
-                        }
-                        const int v0 = (t_begin + j) * kTileN;
-                        const uint32_t sW = sStage + stage * kStageBytes;
-                        const uint32_t sU = sW + kW2Bytes;
-                        mbar_arrive_expect_tx(bar_full + 8 * stage, tx);
-                        tma_load_2d(sW, &tm_w2, bar_full + 8 * stage, v0, 0, pol_w2);
-                        tma_load_3d(sU, &tm_u, bar_full + 8 * stage, v0, k - 1, mt * kMTile, pol_u);
-                        ++issued;
-                        if (++stage == kStages) {
-                            stage = 0;
-                            phase ^= 1u;
+                    for (int t = 0; t < ntiles && ok; ++t) {
+                        int first, count;
+                        tile_span(t, n_units, ntiles, first, count);
+                        const int v0 = (u_begin + first) * kUnit;
+                        const int nbox = (count + 1) >> 1;
+                        for (int ks = 0; ks < kKSlices; ++ks) {
+                            if (!wait_phase(bar_w2_empty + 8 * w2.slot, w2.phase ^ 1u, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t bar = bar_w2_full + 8 * w2.slot;
+                            const uint32_t dst = sW2 + w2.slot * kW2StageBytes;
+                            mbar_arrive_expect_tx(bar, nbox * kW2BoxBytes);
+                            for (int i = 0; i < nbox; ++i)
+                                tma_load_2d(dst + i * kW2BoxBytes, &tm_w2, bar, v0 + 64 * i,
+                                            ks * kKSlice, pol_w2);
+                            ++issued;
+                            w2.next(p.w2_stages);
                         }
                     }
                 }
             }
-            // every issued copy must land before the CTA may exit
-            for (int s = 0; s < kStages; ++s) {
-                const long long uses = issued / kStages + (s < issued % kStages ? 1 : 0);
-                if (uses > 0) wait_drain(bar_full + 8 * s, static_cast<uint32_t>((uses - 1) & 1), p);
-            }
+            drain_ring(bar_w2_full, p.w2_stages, issued, p);   // copies must land before exit
         }
-    } else if (warp == 5) {
+    } else if (warp == kWarpU) {
+        // ------------------------------------------------------------ U producer
+        if (lane == 0) {
+            const uint64_t pol_u = l2_policy_evict_first();
+            const uint32_t u_tx = static_cast<uint32_t>(p.ub) * kUnit * 2;
+            Ring ur;
+            long long issued = 0;
+            bool ok = true;
+            for (int k = 1; k <= p.gamma && ok; ++k) {
+                for (int mt = 0; mt < num_mt && ok; ++mt) {
+                    for (int t = 0; t < ntiles && ok; ++t) {
+                        int first, count;
+                        tile_span(t, n_units, ntiles, first, count);
+                        const int v0 = (u_begin + first) * kUnit;
+                        for (int u = 0; u < count; ++u) {
+                            if (!wait_phase(bar_u_empty + 8 * ur.slot, ur.phase ^ 1u, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t bar = bar_u_full + 8 * ur.slot;
+                            mbar_arrive_expect_tx(bar, u_tx);
+                            tma_load_3d(sU + ur.slot * p.u_slot_bytes, &tm_u, bar, v0 + u * kUnit,
+                                        k - 1, mt * M, pol_u);
+                            ++issued;
+                            ur.next(p.u_slots);
+                        }
+                    }
+                }
+            }
+            drain_ring(bar_u_full, p.u_slots, issued, p);
+        }
+    } else if (warp == kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kMTile, kTileN, 1);
-            int stage = 0;
-            uint32_t phase = 0;
-            int acc = 0;
-            uint32_t aphase = 0;
+            Ring w2, acc, ur;
+            const uint32_t idesc_u = idesc_bf16_f32(static_cast<uint32_t>(M), kUnit, 1);
             uint32_t mt_count = 0;
             bool issued_any = false;
             bool ok = true;
@@ -295,33 +449,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    for (int j = 0; j < ntiles; ++j) {
-                        if (!wait_phase(bar_full + 8 * stage, phase, ctl, p) ||
-                            !wait_phase(bar_tempty + 8 * acc, aphase ^ 1u, ctl, p)) {
+                    for (int t = 0; t < ntiles && ok; ++t) {
+                        int first, count;
+                        tile_span(t, n_units, ntiles, first, count);
+                        const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(M),
+                                                              static_cast<uint32_t>(count * kUnit), 1);
+                        if (!wait_phase(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kTileN);
-                        const uint32_t sW = sStage + stage * kStageBytes;
+                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * 256);
+                        for (int ks = 0; ks < kKSlices; ++ks) {
+                            if (!wait_phase(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t sB = sW2 + w2.slot * kW2StageBytes;
 #pragma unroll
-                        for (int kk = 0; kk < kRank / 16; ++kk) {
-                            const uint64_t a_desc = smem_desc(
-                                sA + (kk >> 2) * kAChunk + (kk & 3) * 32, 1024, 1024, kSwizzle128B);
-                            const uint64_t b_desc = smem_desc(sW + kk * 1024, 512, 512, kSwizzle64B);
-                            umma_bf16(d_tmem, a_desc, b_desc, idesc, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < kKSlice / 16; ++kk) {
+                                const uint64_t a_desc =
+                                    smem_desc(sA + ks * a_chunk + kk * 32, 1024, 1024, kSwizzle128B);
+                                const uint64_t b_desc =
+                                    smem_desc(sB + kk * 2048, kW2BoxBytes, 1024, kSwizzle128B);
+                                umma_bf16(d_tmem, a_desc, b_desc, idesc, (ks | kk) ? 1u : 0u);
+                            }
+                            issued_any = true;
+                            umma_commit(bar_w2_empty + 8 * w2.slot);
+                            w2.next(p.w2_stages);
                         }
-                        issued_any = true;
-                        umma_commit(bar_tfull + 8 * acc);
-                        umma_commit(bar_empty + 8 * stage);
-                        if (++stage == kStages) {
-                            stage = 0;
-                            phase ^= 1u;
+                        if (!ok) break;
+                        // + U_k: D[:, 32u .. 32u + 31] += U_tile(u) x I (two K = 16 halves)
+                        for (int u = 0; u < count; ++u) {
+                            if (!wait_phase(bar_u_full + 8 * ur.slot, ur.phase, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t sUt = sU + ur.slot * p.u_slot_bytes;
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint64_t a_desc = smem_desc(sUt + 32 * h, 512, 512, kSwizzle64B);
+                                const uint64_t b_desc = smem_desc(sI + 1024 * h, 512, 512, kSwizzle64B);
+                                umma_bf16(d_tmem + static_cast<uint32_t>(u * kUnit), a_desc, b_desc,
+                                          idesc_u, 1u);
+                            }
+                            umma_commit(bar_u_empty + 8 * ur.slot);
+                            ur.next(p.u_slots);
                         }
-                        if (++acc == kAcc) {
-                            acc = 0;
-                            aphase ^= 1u;
-                        }
+                        if (!ok) break;
+                        umma_commit(bar_tfull + 8 * acc.slot);
+                        acc.next(kAcc);
                     }
                     if (!ok) break;
                     umma_commit(bar_aempty);
@@ -334,164 +513,99 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue (warps 0-3)
-        const int row = warp * 32 + lane;
-        const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        int stage = 0;
-        uint32_t phase = 0;
-        int acc = 0;
-        uint32_t aphase = 0;
+        // ------------------------------------------------------------ epilogue (warps 0-7)
+        const int q = warp & 3;                   // TMEM lane quadrant
+        const int half = warp >> 2;               // which 32-column chunks of a tile
+        const int rq = M / 4;                     // rows per quadrant: 16 or 32
+        const bool lane_row = lane < rq;
+        const int row = q * rq + lane;            // row of the M tile held by this lane
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        const int chunk = lane >> 3, unit = lane & 7;
+        const int gather_rows = rq / 2;           // rows of the quadrant this warp gathers
+        Ring acc;
         uint32_t mt_count = 0;
         bool ok = true;
+        int next_tok[kMaxMTiles];
+        unsigned long long my_key[kMaxMTiles];
+        float my_logit[kMaxMTiles];
+        for (int mt = 0; mt < num_mt; ++mt) {
+            const int b = mt * M + row;
+            next_tok[mt] = (lane_row && b < p.B) ? checked_token(p.anchor[b], p.V) : -1;
+        }
 
         for (int k = 1; k <= p.gamma && ok; ++k) {
             for (int mt = 0; mt < num_mt && ok; ++mt) {
-                const int m0 = mt * kMTile;
-                // ---- gather A = W1[x_{k-1}] for this block of requests (K-major, 128B swizzle)
-                if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
+                const int m0 = mt * M;
+                const int my_b = m0 + row;
+                // ---- gather A = W1[x_{k-1}] (K-major, 128-byte swizzle), all rows in flight
+                if (!__all_sync(0xFFFFFFFFu,
+                                wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
                     ok = false;
                     break;
                 }
-                const int my_b = m0 + row;
-                const int my_tok = (my_b < p.B) ? prev_token(p, my_b, k) : -1;
-                const int chunk = lane >> 3, unit = lane & 7;
-#pragma unroll 1
-                for (int i0 = 0; i0 < 32; i0 += 8) {
-                    int4 v[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int tok = __shfl_sync(0xFFFFFFFFu, my_tok, i0 + q);
-                        if (tok >= 0) {
-                            v[q] = __ldg(reinterpret_cast<const int4 *>(
-                                p.W1 + static_cast<size_t>(tok) * kRank + lane * 8));
-                        } else {
-                            v[q] = make_int4(0, 0, 0, 0);
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int r = warp * 32 + i0 + q;
-                        sts128(sA + chunk * kAChunk + r * 128 + ((unit ^ (r & 7)) << 4), v[q]);
-                    }
+                const int my_tok = next_tok[mt];
+                for (int i = 0; i < gather_rows; ++i) {
+                    const int src_lane = half * gather_rows + i;
+                    const int tok = __shfl_sync(0xFFFFFFFFu, my_tok, src_lane);
+                    const int r = q * rq + src_lane;
+                    const uint32_t dst = sA + chunk * a_chunk + r * 128 + ((unit ^ (r & 7)) << 4);
+                    if (tok >= 0)
+                        cp_async_16(dst, p.W1 + static_cast<size_t>(tok) * kRank + lane * 8);
+                    else
+                        sts128_zero(dst);
                 }
+                cp_async_wait_all();
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_afull);
                 ++mt_count;
 
-                // ---- vocabulary tiles of this CTA
-                const bool active = (m0 + warp * 32) < p.B;
+                // ---- vocabulary tiles of this CTA: this warp takes chunks u with u % 2 == half
+                const bool active = (m0 + q * rq) < p.B;
                 const int b_glob = my_b + p.b_offset;
-                float best_s = -INFINITY, best_l = 0.0f;
-                uint32_t best_v = 0xFFFFFFFFu;
-                for (int j = 0; j < ntiles; ++j) {
+                RowBest best;
+                for (int t = 0; t < ntiles && ok; ++t) {
+                    int first, count;
+                    tile_span(t, n_units, ntiles, first, count);
                     // warp-uniform outcome: tcgen05.ld below needs every lane of the warp
-                    if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_tfull + 8 * acc, aphase, ctl, p))) {
+                    if (!__all_sync(0xFFFFFFFFu,
+                                    wait_phase(bar_tfull + 8 * acc.slot, acc.phase, ctl, p))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    // this warp's chunks: u = half, half + 2, ...
+                    const int nmine = count > half ? (count - half + 1) / 2 : 0;
+                    const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * 256);
                     if (active) {
-                        uint32_t a[32];
-                        tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(acc * kTileN), a);
-                        tmem_wait_ld();
-                        const uint32_t sU = sStage + stage * kStageBytes + kW2Bytes;
-                        const int v0 = (t_begin + j) * kTileN;
-                        float l[32];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            uint32_t w0, w1, w2, w3;
-                            lds128(sU + row * 64 + ((u ^ ((row >> 1) & 3)) << 4), w0, w1, w2, w3);
-                            l[8 * u + 0] = __uint_as_float(a[8 * u + 0]) + bf16lo_to_f32(w0);
-                            l[8 * u + 1] = __uint_as_float(a[8 * u + 1]) + bf16hi_to_f32(w0);
-                            l[8 * u + 2] = __uint_as_float(a[8 * u + 2]) + bf16lo_to_f32(w1);
-                            l[8 * u + 3] = __uint_as_float(a[8 * u + 3]) + bf16hi_to_f32(w1);
-                            l[8 * u + 4] = __uint_as_float(a[8 * u + 4]) + bf16lo_to_f32(w2);
-                            l[8 * u + 5] = __uint_as_float(a[8 * u + 5]) + bf16hi_to_f32(w2);
-                            l[8 * u + 6] = __uint_as_float(a[8 * u + 6]) + bf16lo_to_f32(w3);
-                            l[8 * u + 7] = __uint_as_float(a[8 * u + 7]) + bf16hi_to_f32(w3);
-                        }
-                        if (v0 + kTileN > p.V) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (v0 + i >= p.V) l[i] = -INFINITY;
-                        }
-                        float s[32];
-                        if (p.mode == 0) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) s[i] = l[i];
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float lmax = fmaxf(fmaxf(l[4 * q], l[4 * q + 1]),
-                                                         fmaxf(l[4 * q + 2], l[4 * q + 3]));
-                                // noise cannot lift this group above the running best
-                                const bool skip =
-                                    !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best_s);
-                                if (__all_sync(0xFFFFFFFFu, skip)) {
-                                    s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
-                                } else {
-                                    const uint4 w = philox(
-                                        make_uint4(static_cast<uint32_t>(v0 / 4 + q),
-                                                   static_cast<uint32_t>(k - 1),
-                                                   static_cast<uint32_t>(b_glob), 0u),
-                                        p.seed_lo, p.seed_hi);
-                                    s[4 * q + 0] = fmaf(l[4 * q + 0], p.inv_tau, gumbel_from_word(w.x));
-                                    s[4 * q + 1] = fmaf(l[4 * q + 1], p.inv_tau, gumbel_from_word(w.y));
-                                    s[4 * q + 2] = fmaf(l[4 * q + 2], p.inv_tau, gumbel_from_word(w.z));
-                                    s[4 * q + 3] = fmaf(l[4 * q + 3], p.inv_tau, gumbel_from_word(w.w));
-                                    if (skip) s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
-                                }
-                            }
-                        }
-                        float mx = s[0];
-#pragma unroll
-                        for (int i = 1; i < 32; ++i) mx = fmaxf(mx, s[i]);
-                        if (mx > best_s) {
-                            int idx = 31;
-#pragma unroll
-                            for (int i = 31; i >= 0; --i)
-                                if (s[i] == mx) idx = i;
-                            best_s = mx;
-                            best_v = static_cast<uint32_t>(v0 + idx);
-                            float li = l[0];
-#pragma unroll
-                            for (int i = 1; i < 32; ++i)
-                                if (i == idx) li = l[i];
-                            best_l = li;
+                        for (int jj = 0; jj < nmine; ++jj) {
+                            const int u = half + 2 * jj;
+                            uint32_t a[32];
+                            tmem_ld_32x32b_x32(t_acc + u * kUnit, a);
+                            tmem_wait_ld();
+                            chunk_update(best, a, (u_begin + first + u) * kUnit, p, k, b_glob);
                         }
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(bar_tempty + 8 * acc);
-                        mbar_arrive(bar_empty + 8 * stage);
-                    }
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                    if (++acc == kAcc) {
-                        acc = 0;
-                        aphase ^= 1u;
-                    }
+                    if (lane == 0) mbar_arrive(bar_tempty + 8 * acc.slot);
+                    acc.next(kAcc);
                 }
                 if (!ok) break;
-                if (my_b < p.B) {
-                    const unsigned long long key = argmax_key(best_s, best_v);
+                if (lane_row && my_b < p.B) {
+                    const unsigned long long key = argmax_key(best.s, best.v);
                     atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + my_b], key);
-                    row_key[my_b] = key;
-                    row_logit[my_b] = best_l;
+                    my_key[mt] = key;
+                    my_logit[mt] = best.l;
                 }
             }
 
             // ---- grid barrier: every CTA has combined its rows of position k
             epi_sync();
             if (threadIdx.x == 0 && ok && !*reinterpret_cast<volatile int *>(&ctl.abort)) {
-                __threadfence();
-                atomicAdd(p.barrier, 1u);
-                const uint32_t target =
-                    static_cast<uint32_t>(k) * static_cast<uint32_t>(G) + static_cast<uint32_t>(p.barrier_extra);
+                red_release_add_u32(p.barrier, 1u);
+                const uint32_t target = static_cast<uint32_t>(k) * static_cast<uint32_t>(G) +
+                                        static_cast<uint32_t>(p.barrier_extra);
                 const uint64_t t0 = globaltimer_ns();
                 while (ld_acquire_u32(p.barrier) < target) {
                     if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
@@ -502,23 +616,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         give_up(ctl, p, DSPARK_TIMEOUT);
                         break;
                     }
-                    __nanosleep(64);
+                    __nanosleep(32);
                 }
-                __threadfence();
             }
             epi_sync();
             if (!ok || *reinterpret_cast<volatile int *>(&ctl.abort)) {
                 ok = false;
                 break;
             }
-            // ---- outputs of position k: written by the CTA that owns the winning column
-            for (int b = threadIdx.x; b < p.B; b += kEpiThreads) {
-                const unsigned long long key =
-                    __ldcg(&p.slots[static_cast<size_t>(k - 1) * p.B + b]);
-                if (key == row_key[b]) {
-                    p.x_out[static_cast<size_t>(b) * p.gamma + (k - 1)] =
-                        static_cast<int32_t>(argmax_key_index(key));
-                    p.logit_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = row_logit[b];
+            // ---- x_k of my rows: next gather's tokens; the owning CTA/half writes the outputs
+            for (int mt = 0; mt < num_mt; ++mt) {
+                const int b = mt * M + row;
+                if (!lane_row || b >= p.B) continue;
+                const size_t o = static_cast<size_t>(k - 1) * p.B + b;
+                const unsigned long long key = __ldcg(&p.slots[o]);
+                const int tok = static_cast<int>(argmax_key_index(key));
+                next_tok[mt] = checked_token(tok, p.V);
+                if (key == my_key[mt]) {
+                    p.x_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = tok;
+                    p.logit_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = my_logit[mt];
                 }
             }
         }
@@ -526,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
