@@ -152,6 +152,32 @@ int dspark_verify_prefix(const int32_t *x, const int32_t *L, const int32_t *targ
                          int gamma, int32_t *accepted_out, int32_t *bonus_out,
                          dspark_stream_t stream);
 
+/*
+ * The prefix scheduler for callers that cannot allocate device memory.
+ * (No counterpart on the DSpark pages: this is an interface convenience.)
+ *
+ * Same arguments, results and error behaviour as dspark_schedule_prefix, minus the
+ * workspace.  It is meant for callers that have no way to hand the library a workspace:
+ * processes whose device memory is fixed when they start (a serving engine that divides
+ * all of HBM into its own pools, an embedded runtime with a set memory budget), or code
+ * that must not call cudaMalloc at this point because the call can synchronise the device
+ * and stall other streams.  The library calls no allocating routine here either.
+ *
+ * Scratch lives in one statically sized array inside this library's device image
+ * (288 KB, held by every GPU that loads the library until the process exits), so:
+ *   - B * gamma must not exceed 24576; larger sizes return DSPARK_UNSUPPORTED_SHAPE;
+ *   - every call on a device shares that array, and the array keeps the last call's
+ *     contents: calls that can overlap on the GPU (different streams, or different host
+ *     threads without ordering between their streams) race and give wrong results;
+ *     order them on one stream;
+ *   - the first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture.
+ */
+int dspark_schedule_prefix_noalloc(const float *P, int B, int gamma, const double *Tstep_us,
+                                   int32_t *L_out, int32_t *N_out, double *objective_out,
+                                   dspark_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device into *status (DSPARK_OK when nothing was recorded). */
 int dspark_get_error(dspark_stream_t stream, int *status);

@@ -313,6 +313,85 @@ int dspark_verify_prefix(const int32_t *x, const int32_t *L, const int32_t *targ
     return from_cuda(cudaGetLastError());
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Scheduler entry point for callers that cannot allocate device memory.
+//
+// dspark_schedule_prefix needs a caller-provided workspace.  Some callers have no way
+// to provide one: their device memory is fixed when the process starts (a serving
+// engine that carves all of HBM into its own pools, an embedded runtime with a set
+// budget), or they must not call cudaMalloc on this path because it can synchronise
+// the device and stall other streams.  This variant keeps its scratch in the static
+// array below instead, which is part of this library's device image: every GPU that
+// loads the library holds it (288 KB) until the process exits.
+namespace {
+
+constexpr int kNoAllocMaxScores = 24576;                          // B * gamma limit
+constexpr size_t kNoAllocRankOffset = kCtlBytes;
+constexpr size_t kNoAllocQOffset = kCtlBytes + static_cast<size_t>(kNoAllocMaxScores) * 4;
+constexpr size_t kNoAllocScratchBytes = kNoAllocQOffset + static_cast<size_t>(kNoAllocMaxScores) * 8;
+
+static __device__ __align__(256) unsigned char g_sched_scratch[kNoAllocScratchBytes];
+
+// Device address of g_sched_scratch per device (0 until that device's first call).
+// In host code the symbol names only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress while the device is current.
+void *g_sched_scratch_dev[kMaxDevices];
+
+}  // namespace
+
+extern "C" {
+
+int dspark_schedule_prefix_noalloc(const float *P, int B, int gamma, const double *Tstep_us,
+                                   int32_t *L_out, int32_t *N_out, double *objective_out,
+                                   dspark_stream_t stream)
+{
+    namespace S = dspark::sched;
+    if (!P || !Tstep_us || !L_out || !N_out || !objective_out) return DSPARK_INVALID_ARG;
+    if (!aligned(P, 4) || !aligned(Tstep_us, 8) || !aligned(L_out, 4) || !aligned(N_out, 4) ||
+        !aligned(objective_out, 8))
+        return DSPARK_INVALID_ARG;
+    if (B < 1 || gamma < 1 || gamma > 64 ||
+        static_cast<long long>(B) * gamma > kNoAllocMaxScores)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    DeviceInfo *dev = nullptr;
+    if (int st = current_device(&dev)) return st;
+    int dev_id = 0;
+    if (cudaGetDevice(&dev_id) != cudaSuccess) return DSPARK_CUDA_ERROR;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        if (!g_sched_scratch_dev[dev_id]) {
+            void *addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_sched_scratch) != cudaSuccess || !addr)
+                return DSPARK_CUDA_ERROR;
+            g_sched_scratch_dev[dev_id] = addr;
+        }
+        scratch = g_sched_scratch_dev[dev_id];
+    }
+    uint8_t *ws = static_cast<uint8_t *>(scratch);
+    const int n = B * gamma;
+    S::Params prm;
+    prm.P = P;
+    prm.B = B;
+    prm.gamma = gamma;
+    prm.n = n;
+    prm.Tstep = Tstep_us;
+    prm.L_out = L_out;
+    prm.N_out = N_out;
+    prm.objective_out = objective_out;
+    prm.done = reinterpret_cast<unsigned int *>(ws);
+    prm.rank = reinterpret_cast<int32_t *>(ws + kNoAllocRankOffset);
+    prm.q_sorted = reinterpret_cast<long long *>(ws + kNoAllocQOffset);
+    // the completion counter must start at zero; the rest is fully rewritten by the kernel
+    if (cudaMemsetAsync(ws, 0, kCtlBytes, stream) != cudaSuccess) return DSPARK_CUDA_ERROR;
+    int grid = (n + S::kWarps - 1) / S::kWarps;
+    if (grid > 2 * dev->sms) grid = 2 * dev->sms;
+    S::schedule_prefix_kernel<<<grid, S::kThreads, 0, stream>>>(prm);
+    return from_cuda(cudaGetLastError());
+}
+
 int dspark_get_error(dspark_stream_t stream, int *status)
 {
     if (!status) return DSPARK_INVALID_ARG;
