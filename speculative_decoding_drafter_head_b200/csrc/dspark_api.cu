@@ -174,10 +174,10 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
                                     static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(V) * 2,
                                        static_cast<cuuint64_t>(V) * 2 * gamma};
-        const cuuint32_t box[3] = {D::kUnit, 1, static_cast<cuuint32_t>(ub)};
+        const cuuint32_t box[3] = {D::kUBoxCols, 1, static_cast<cuuint32_t>(ub)};
         const cuuint32_t estr[3] = {1, 1, 1};
         if (encode(&tm_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(U), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return DSPARK_CUDA_ERROR;
@@ -212,7 +212,7 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     prm.M = M;
     prm.w2_stages = M == 64 ? 4 : 3;
     prm.ub = ub;
-    prm.u_slot_bytes = M * D::kUnit * 2;   // a full M-row tile: the MMA reads all M rows
+    prm.u_slot_bytes = static_cast<int>(round_up(static_cast<size_t>(ub) * D::kUBoxCols * 2, 1024));
     prm.u_slots = D::kURingBytes / prm.u_slot_bytes;
     if (prm.u_slots > D::kUMaxSlots) prm.u_slots = D::kUMaxSlots;
     prm.timeout_ns = g_timeout_ns.load();

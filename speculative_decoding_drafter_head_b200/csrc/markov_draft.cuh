@@ -10,13 +10,13 @@
 // over the grid) cut into tiles of up to 256 columns, and for every position k and
 // every block of M requests it computes
 //     D[b, v] = sum_j A[b, j] W2[j, v],   A[b, :] = W1[x_{k-1, b}, :]
-// as tcgen05.mma M=64/128, N<=256, K=16 (bf16 in, fp32 accumulate in TMEM), with W2
-// streamed by TMA in four K-slices of 64 rows (MN-major, 128-byte swizzle).  U_k is
-// added on the tensor core as well: each 32-column U tile, as staged by TMA (K-major,
-// 64-byte swizzle), is multiplied by a 32 x 32 identity into the same accumulator,
-// which is exact (bf16 times 1 into fp32).  The epilogue therefore reads finished
-// logits from TMEM, applies greedy or Gumbel-max selection and keeps a running
-// (max, index) per request row, so the [B, V] logits never reach memory.  Rows are
+// as tcgen05.mma M=64/128, N<=128, K=16 (bf16 in, fp32 accumulate in TMEM), with W2
+// streamed by TMA in two K-halves of 128 rows (MN-major, 128-byte swizzle).  A single
+// MMA instruction costs the same for any N up to 128 and for M = 64 or 128, so tiles
+// are 128 columns wide and a CTA's odd remainder becomes one narrow tile.  The
+// epilogue adds U_k (staged by TMA), applies greedy or Gumbel-max selection and keeps
+// a running (max, index) per request row, so the [B, V] logits never reach memory.
+// Rows are
 // combined across CTAs by a 64-bit atomicMax on (ordered value, inverted index); a
 // bounded grid barrier ends each position, after which every CTA reads x_k for the
 // next gather and the CTA that owns the winning column writes the outputs.
@@ -37,20 +37,21 @@
 namespace dspark {
 namespace draft {
 
-constexpr int kUnit = 32;                         // columns per U box and epilogue chunk
-constexpr int kMaxUnits = 8;                      // 256 columns per MMA tile
+constexpr int kUnit = 32;                         // columns per epilogue chunk
+constexpr int kUBoxCols = 64;                     // columns per U TMA box (two chunks)
+constexpr int kMaxUnits = 4;                      // 128 columns per MMA tile
 constexpr int kRank = 256;                        // r, the contraction length
-constexpr int kKSlice = 64;                       // W2 rows per ring stage
-constexpr int kKSlices = kRank / kKSlice;         // 4
+constexpr int kKSlice = 128;                      // W2 rows per ring stage
+constexpr int kKSlices = kRank / kKSlice;         // 2
 constexpr int kMaxW2Stages = 4;
-constexpr int kW2BoxBytes = 64 * kKSlice * 2;     // one TMA box: 64 columns x 64 rows
-constexpr int kW2StageBytes = 4 * kW2BoxBytes;    // 32 KB: 256 columns x 64 rows
-constexpr int kURingBytes = 62 * 1024;            // U tiles, M rows x 32 columns each
+constexpr int kW2BoxBytes = 64 * kKSlice * 2;     // one TMA box: 64 columns x 128 rows (16 KB)
+constexpr int kW2StageBytes = 2 * kW2BoxBytes;    // 32 KB: 128 columns x 128 rows
+constexpr int kURingBytes = 64 * 1024;            // U boxes, rows x 64 columns each
 constexpr int kUMaxSlots = 16;
-constexpr int kIdentBytes = 2 * 1024;             // 32 x 32 bf16 identity (B operand)
-constexpr int kAcc = 2;                           // TMEM accumulators of 256 columns
+constexpr int kAcc = 4;                           // TMEM accumulators of 128 columns
+constexpr int kAccCols = 128;
 constexpr uint32_t kTmemCols = 512;
-// A (M x 256 bf16) + W2 ring + U ring + identity: M = 64 with 4 W2 stages or M = 128 with 3
+// A (M x 256 bf16) + W2 ring + U ring: M = 64 with 4 W2 stages or M = 128 with 3
 constexpr int kDynSmem = 224 * 1024 + 1024;       // + alignment slack
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
 constexpr int kThreads = (kEpiWarps + 3) * 32;    // + W2 producer, U producer, MMA issuer
@@ -76,7 +77,7 @@ struct Params {
     int M;                       // requests per MMA tile: 64 (B <= 64) or 128
     int w2_stages;               // W2 ring depth (4 when M = 64, else 3)
     int ub;                      // rows of the U TMA box: min(B, M)
-    int u_slots;                 // U ring depth
+    int u_slots;                 // U ring depth (boxes of 64 columns)
     int u_slot_bytes;
     unsigned long long timeout_ns;
     int barrier_extra;
@@ -107,12 +108,13 @@ struct Ring {
     }
 };
 
-// The t-th tile of a CTA that owns n_units units split into ntiles balanced tiles.
+// The t-th tile of a CTA that owns n_units units: full tiles of kMaxUnits units, then
+// the remainder (an MMA costs the same for any N <= 128, so this minimises the count).
 __device__ __forceinline__ void tile_span(int t, int n_units, int ntiles, int &first, int &count)
 {
-    const int base = n_units / ntiles, extra = n_units % ntiles;
-    first = t * base + min(t, extra);
-    count = base + (t < extra ? 1 : 0);
+    (void)ntiles;
+    first = t * kMaxUnits;
+    count = min(kMaxUnits, n_units - first);
 }
 
 __device__ __forceinline__ void give_up(Ctl &ctl, const Params &p, unsigned code)
@@ -232,15 +234,36 @@ __device__ __forceinline__ float max32(const float (&s)[32])
     return fmaxf(fmax3(a, b, c), d);
 }
 
-// Running best of one request row over one 32-column chunk of finished logits l
-// (U_k + bias, from TMEM): greedy or Gumbel-max score s; a strict improvement keeps
-// the smallest column on ties.
-__device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[32], int v0,
-                                             const Params &p, int k, int b_glob)
+__device__ __forceinline__ void lds128(uint32_t addr, uint32_t &a, uint32_t &b, uint32_t &c,
+                                       uint32_t &d)
+{
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+                 : "r"(addr));
+}
+
+// Running best of one request row over one 32-column chunk: l = acc + U, where the U
+// row sits in a 64-column box in shared memory (128-byte rows, 128-byte swizzle) and the
+// chunk is its columns 32 h .. 32 h + 31; greedy or Gumbel-max score s; a strict
+// improvement keeps the smallest column on ties.
+__device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[32], uint32_t sU,
+                                             int row, int h, int v0, const Params &p, int k,
+                                             int b_glob)
 {
     float l[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) l[i] = __uint_as_float(a[i]);
+    for (int u = 0; u < 4; ++u) {
+        uint32_t w0, w1, w2, w3;
+        lds128(sU + row * 128 + (((4 * h + u) ^ (row & 7)) << 4), w0, w1, w2, w3);
+        l[8 * u + 0] = __uint_as_float(a[8 * u + 0]) + bf16lo_to_f32(w0);
+        l[8 * u + 1] = __uint_as_float(a[8 * u + 1]) + bf16hi_to_f32(w0);
+        l[8 * u + 2] = __uint_as_float(a[8 * u + 2]) + bf16lo_to_f32(w1);
+        l[8 * u + 3] = __uint_as_float(a[8 * u + 3]) + bf16hi_to_f32(w1);
+        l[8 * u + 4] = __uint_as_float(a[8 * u + 4]) + bf16lo_to_f32(w2);
+        l[8 * u + 5] = __uint_as_float(a[8 * u + 5]) + bf16hi_to_f32(w2);
+        l[8 * u + 6] = __uint_as_float(a[8 * u + 6]) + bf16lo_to_f32(w3);
+        l[8 * u + 7] = __uint_as_float(a[8 * u + 7]) + bf16hi_to_f32(w3);
+    }
     if (v0 + kUnit > p.V) {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
@@ -303,7 +326,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sA = base;
     const uint32_t sW2 = base + static_cast<uint32_t>(M * kRank * 2);
     const uint32_t sU = sW2 + static_cast<uint32_t>(p.w2_stages * kW2StageBytes);
-    const uint32_t sI = sU + kURingBytes;
 
     const int G = gridDim.x;
     const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.units_total / G);
@@ -330,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < p.u_slots; ++s) {
             mbar_init(bar_u_full + 8 * s, 1);
-            mbar_init(bar_u_empty + 8 * s, 1);
+            mbar_init(bar_u_empty + 8 * s, kEpiWarps);
         }
         for (int a = 0; a < kAcc; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
@@ -341,21 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar_drain, 1);
         ctl.abort = 0;
         mbar_fence_init();
-    }
-    if (threadIdx.x < 128) {
-        // 32 x 32 identity as an MN-major, 64-byte-swizzled B operand: row k holds 1.0
-        // at column k; 16-byte unit j of row k sits at unit j ^ ((k >> 1) & 3).
-        const int kr = threadIdx.x >> 2, j = threadIdx.x & 3;
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        if (j == (kr >> 3)) {
-            const int e = kr & 7;                         // element within the unit
-            w[e >> 1] = (e & 1) ? 0x3F800000u : 0x00003F80u;
-        }
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                         sI + kr * 64 + ((j ^ ((kr >> 1) & 3)) << 4)),
-                     "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
-                     : "memory");
-        fence_proxy_async_smem();
     }
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
@@ -383,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         int first, count;
                         tile_span(t, n_units, ntiles, first, count);
                         const int v0 = (u_begin + first) * kUnit;
-                        const int nbox = (count + 1) >> 1;
+                        const int nbox = (count + 1) >> 1;          // 64-column boxes
                         for (int ks = 0; ks < kKSlices; ++ks) {
                             if (!wait_phase(bar_w2_empty + 8 * w2.slot, w2.phase ^ 1u, ctl, p)) {
                                 ok = false;
@@ -407,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ U producer
         if (lane == 0) {
             const uint64_t pol_u = l2_policy_evict_first();
-            const uint32_t u_tx = static_cast<uint32_t>(p.ub) * kUnit * 2;
+            const uint32_t u_tx = static_cast<uint32_t>(p.ub) * kUBoxCols * 2;
             Ring ur;
             long long issued = 0;
             bool ok = true;
@@ -417,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         int first, count;
                         tile_span(t, n_units, ntiles, first, count);
                         const int v0 = (u_begin + first) * kUnit;
-                        for (int u = 0; u < count; ++u) {
+                        for (int u = 0; u < count; u += 2) {
                             if (!wait_phase(bar_u_empty + 8 * ur.slot, ur.phase ^ 1u, ctl, p)) {
                                 ok = false;
                                 break;
@@ -437,8 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            Ring w2, acc, ur;
-            const uint32_t idesc_u = idesc_bf16_f32(static_cast<uint32_t>(M), kUnit, 1);
+            Ring w2, acc;
             uint32_t mt_count = 0;
             bool issued_any = false;
             bool ok = true;
@@ -459,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * 256);
+                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
                         for (int ks = 0; ks < kKSlices; ++ks) {
                             if (!wait_phase(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
                                 ok = false;
@@ -469,8 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t sB = sW2 + w2.slot * kW2StageBytes;
 #pragma unroll
                             for (int kk = 0; kk < kKSlice / 16; ++kk) {
-                                const uint64_t a_desc =
-                                    smem_desc(sA + ks * a_chunk + kk * 32, 1024, 1024, kSwizzle128B);
+                                const uint64_t a_desc = smem_desc(
+                                    sA + (2 * ks + (kk >> 2)) * a_chunk + (kk & 3) * 32, 1024, 1024,
+                                    kSwizzle128B);
                                 const uint64_t b_desc =
                                     smem_desc(sB + kk * 2048, kW2BoxBytes, 1024, kSwizzle128B);
                                 umma_bf16(d_tmem, a_desc, b_desc, idesc, (ks | kk) ? 1u : 0u);
@@ -480,24 +487,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             w2.next(p.w2_stages);
                         }
                         if (!ok) break;
-                        // + U_k: D[:, 32u .. 32u + 31] += U_tile(u) x I (two K = 16 halves)
-                        for (int u = 0; u < count; ++u) {
-                            if (!wait_phase(bar_u_full + 8 * ur.slot, ur.phase, ctl, p)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint32_t sUt = sU + ur.slot * p.u_slot_bytes;
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const uint64_t a_desc = smem_desc(sUt + 32 * h, 512, 512, kSwizzle64B);
-                                const uint64_t b_desc = smem_desc(sI + 1024 * h, 512, 512, kSwizzle64B);
-                                umma_bf16(d_tmem + static_cast<uint32_t>(u * kUnit), a_desc, b_desc,
-                                          idesc_u, 1u);
-                            }
-                            umma_commit(bar_u_empty + 8 * ur.slot);
-                            ur.next(p.u_slots);
-                        }
                         if (!ok) break;
                         umma_commit(bar_tfull + 8 * acc.slot);
                         acc.next(kAcc);
@@ -519,10 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rq = M / 4;                     // rows per quadrant: 16 or 32
         const bool lane_row = lane < rq;
         const int row = q * rq + lane;            // row of the M tile held by this lane
+        const int urow = lane_row ? min(row, p.ub - 1) : 0;   // U tile row (stays in the slot)
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
         const int chunk = lane >> 3, unit = lane & 7;
         const int gather_rows = rq / 2;           // rows of the quadrant this warp gathers
         Ring acc;
+        long long u_pos = 0;                      // U boxes consumed so far
         uint32_t mt_count = 0;
         bool ok = true;
         int next_tok[kMaxMTiles];
@@ -574,18 +565,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    // this warp's chunks: u = half, half + 2, ...
-                    const int nmine = count > half ? (count - half + 1) / 2 : 0;
-                    const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * 256);
-                    if (active) {
-                        for (int jj = 0; jj < nmine; ++jj) {
-                            const int u = half + 2 * jj;
+                    // box i of the tile holds chunks 2i and 2i + 1; this warp takes chunk 2i + half
+                    const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
+                    const int nbox = (count + 1) >> 1;
+                    for (int i = 0; i < nbox; ++i) {
+                        const long long pos = u_pos + i;
+                        const int slot = static_cast<int>(pos % p.u_slots);
+                        const uint32_t par = static_cast<uint32_t>((pos / p.u_slots) & 1);
+                        if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_u_full + 8 * slot, par, ctl, p))) {
+                            ok = false;
+                            break;
+                        }
+                        const int u = 2 * i + half;
+                        if (active && u < count) {
                             uint32_t a[32];
                             tmem_ld_32x32b_x32(t_acc + u * kUnit, a);
                             tmem_wait_ld();
-                            chunk_update(best, a, (u_begin + first + u) * kUnit, p, k, b_glob);
+                            chunk_update(best, a, sU + slot * p.u_slot_bytes, urow, half,
+                                         (u_begin + first + u) * kUnit, p, k, b_glob);
                         }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_u_empty + 8 * slot);
                     }
+                    u_pos += nbox;
+                    if (!ok) break;
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_tempty + 8 * acc.slot);
@@ -616,7 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         give_up(ctl, p, DSPARK_TIMEOUT);
                         break;
                     }
-                    __nanosleep(32);
                 }
             }
             epi_sync();
