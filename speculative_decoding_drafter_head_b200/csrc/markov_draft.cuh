@@ -242,15 +242,11 @@ __device__ __forceinline__ void lds128(uint32_t addr, uint32_t &a, uint32_t &b, 
                  : "r"(addr));
 }
 
-// Running best of one request row over one 32-column chunk: l = acc + U, where the U
-// row sits in a 64-column box in shared memory (128-byte rows, 128-byte swizzle) and the
-// chunk is its columns 32 h .. 32 h + 31; greedy or Gumbel-max score s; a strict
-// improvement keeps the smallest column on ties.
-__device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[32], uint32_t sU,
-                                             int row, int h, int v0, const Params &p, int k,
-                                             int b_glob)
+// l = acc + U for 32 columns: the U row sits in a 64-column box in shared memory
+// (128-byte rows, 128-byte swizzle) and these are its columns 32 h .. 32 h + 31.
+__device__ __forceinline__ void add_u32(float (&l)[32], const uint32_t (&a)[32], uint32_t sU,
+                                        int row, int h)
 {
-    float l[32];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         uint32_t w0, w1, w2, w3;
@@ -264,50 +260,90 @@ __device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[
         l[8 * u + 6] = __uint_as_float(a[8 * u + 6]) + bf16lo_to_f32(w3);
         l[8 * u + 7] = __uint_as_float(a[8 * u + 7]) + bf16hi_to_f32(w3);
     }
+}
+
+// Scores of 32 logits starting at column v0: the logits themselves (greedy) or
+// l / tau + Gumbel noise; columns at or beyond V get -inf.
+__device__ __forceinline__ void scores32(float (&s)[32], float (&l)[32], int v0, const Params &p,
+                                         int k, int b_glob, float best_s)
+{
     if (v0 + kUnit > p.V) {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
             if (v0 + i >= p.V) l[i] = -INFINITY;
     }
-    float s[32];
     if (p.mode == 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[i] = l[i];
-    } else {
+        return;
+    }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float lmax =
-                fmaxf(fmaxf(l[4 * q], l[4 * q + 1]), fmaxf(l[4 * q + 2], l[4 * q + 3]));
-            // exact pruning: noise cannot lift this group above the running best
-            const bool skip = !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best.s);
-            if (__all_sync(0xFFFFFFFFu, skip)) {
-                s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
-            } else {
-                const uint4 w = philox(make_uint4(static_cast<uint32_t>(v0 / 4 + q),
-                                                  static_cast<uint32_t>(k - 1),
-                                                  static_cast<uint32_t>(b_glob), 0u),
-                                       p.seed_lo, p.seed_hi);
-                s[4 * q + 0] = fmaf(l[4 * q + 0], p.inv_tau, gumbel_from_word(w.x));
-                s[4 * q + 1] = fmaf(l[4 * q + 1], p.inv_tau, gumbel_from_word(w.y));
-                s[4 * q + 2] = fmaf(l[4 * q + 2], p.inv_tau, gumbel_from_word(w.z));
-                s[4 * q + 3] = fmaf(l[4 * q + 3], p.inv_tau, gumbel_from_word(w.w));
-                if (skip) s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
-            }
+    for (int q = 0; q < 8; ++q) {
+        const float lmax = fmaxf(fmaxf(l[4 * q], l[4 * q + 1]), fmaxf(l[4 * q + 2], l[4 * q + 3]));
+        // exact pruning: noise cannot lift this group above the running best
+        const bool skip = !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best_s);
+        if (__all_sync(0xFFFFFFFFu, skip)) {
+            s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
+        } else {
+            const uint4 w = philox(make_uint4(static_cast<uint32_t>(v0 / 4 + q),
+                                              static_cast<uint32_t>(k - 1),
+                                              static_cast<uint32_t>(b_glob), 0u),
+                                   p.seed_lo, p.seed_hi);
+            s[4 * q + 0] = fmaf(l[4 * q + 0], p.inv_tau, gumbel_from_word(w.x));
+            s[4 * q + 1] = fmaf(l[4 * q + 1], p.inv_tau, gumbel_from_word(w.y));
+            s[4 * q + 2] = fmaf(l[4 * q + 2], p.inv_tau, gumbel_from_word(w.z));
+            s[4 * q + 3] = fmaf(l[4 * q + 3], p.inv_tau, gumbel_from_word(w.w));
+            if (skip) s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
         }
     }
-    const float mx = max32(s);
+}
+
+// First index of the largest of 32 scores (the caller knows the largest is mx).
+__device__ __forceinline__ int first_index(const float (&s)[32], float mx)
+{
+    int idx = 31;
+#pragma unroll
+    for (int i = 31; i >= 0; --i)
+        if (s[i] == mx) idx = i;
+    return idx;
+}
+
+__device__ __forceinline__ float pick(const float (&l)[32], int idx)
+{
+    float li = l[0];
+#pragma unroll
+    for (int i = 1; i < 32; ++i)
+        if (i == idx) li = l[i];
+    return li;
+}
+
+// Running best of one request row over one 64-column U box: chunk 0 holds columns
+// v0 .. v0 + 31 and, when `two`, chunk 1 holds v0 + 32 .. v0 + 63.  The two 32-column
+// chains are independent until one compare against the running best, which keeps the
+// smallest column on ties.
+__device__ __forceinline__ void box_update(RowBest &best, const uint32_t (&a0)[32],
+                                           const uint32_t (&a1)[32], bool two, uint32_t sU,
+                                           int row, int v0, const Params &p, int k, int b_glob)
+{
+    float l0[32], l1[32], s0[32], s1[32];
+    add_u32(l0, a0, sU, row, 0);
+    add_u32(l1, a1, sU, row, 1);
+    scores32(s0, l0, v0, p, k, b_glob, best.s);
+    scores32(s1, l1, v0 + kUnit, p, k, b_glob, best.s);
+    const float m0 = max32(s0);
+    const float m1 = two ? max32(s1) : -INFINITY;
+    const float mx = fmaxf(m0, m1);
     if (mx > best.s) {
-        int idx = 31;
-#pragma unroll
-        for (int i = 31; i >= 0; --i)
-            if (s[i] == mx) idx = i;
-        float li = l[0];
-#pragma unroll
-        for (int i = 1; i < 32; ++i)
-            if (i == idx) li = l[i];
+        if (m0 == mx) {
+            const int idx = first_index(s0, mx);
+            best.v = static_cast<uint32_t>(v0 + idx);
+            best.l = pick(l0, idx);
+        } else {
+            const int idx = first_index(s1, mx);
+            best.v = static_cast<uint32_t>(v0 + kUnit + idx);
+            best.l = pick(l1, idx);
+        }
         best.s = mx;
-        best.l = li;
-        best.v = static_cast<uint32_t>(v0 + idx);
     }
 }
 
@@ -352,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < p.u_slots; ++s) {
             mbar_init(bar_u_full + 8 * s, 1);
-            mbar_init(bar_u_empty + 8 * s, kEpiWarps);
+            mbar_init(bar_u_empty + 8 * s, kEpiWarps / 2);
         }
         for (int a = 0; a < kAcc; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
@@ -445,6 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             Ring w2, acc;
+            const uint64_t a_desc0 = smem_desc(sA, 1024, 1024, kSwizzle128B);
+            const uint64_t b_desc0 = smem_desc(sW2, kW2BoxBytes, 1024, kSwizzle128B);
             uint32_t mt_count = 0;
             bool issued_any = false;
             bool ok = true;
@@ -472,14 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 break;
                             }
                             tc_fence_after();
-                            const uint32_t sB = sW2 + w2.slot * kW2StageBytes;
+                            // descriptors differ only in the start-address field (bits 0..13,
+                            // 16-byte units): advance them with plain adds
+                            const uint64_t a_k = a_desc0 + static_cast<uint64_t>((2 * ks * a_chunk) >> 4);
+                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((w2.slot * kW2StageBytes) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < kKSlice / 16; ++kk) {
-                                const uint64_t a_desc = smem_desc(
-                                    sA + (2 * ks + (kk >> 2)) * a_chunk + (kk & 3) * 32, 1024, 1024,
-                                    kSwizzle128B);
-                                const uint64_t b_desc =
-                                    smem_desc(sB + kk * 2048, kW2BoxBytes, 1024, kSwizzle128B);
+                                const uint64_t a_desc =
+                                    a_k + static_cast<uint64_t>(((kk >> 2) * a_chunk + (kk & 3) * 32) >> 4);
+                                const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
                                 umma_bf16(d_tmem, a_desc, b_desc, idesc, (ks | kk) ? 1u : 0u);
                             }
                             issued_any = true;
@@ -565,10 +604,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    // box i of the tile holds chunks 2i and 2i + 1; this warp takes chunk 2i + half
+                    // box i of the tile holds chunks 2i and 2i + 1; this warp takes boxes i = half,
+                    // half + 2, ... and reduces both chunks of a box together
                     const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
                     const int nbox = (count + 1) >> 1;
-                    for (int i = 0; i < nbox; ++i) {
+                    for (int i = half; i < nbox; i += 2) {
                         const long long pos = u_pos + i;
                         const int slot = static_cast<int>(pos % p.u_slots);
                         const uint32_t par = static_cast<uint32_t>((pos / p.u_slots) & 1);
@@ -576,13 +616,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        const int u = 2 * i + half;
-                        if (active && u < count) {
-                            uint32_t a[32];
-                            tmem_ld_32x32b_x32(t_acc + u * kUnit, a);
+                        if (active) {
+                            const bool two = 2 * i + 1 < count;
+                            uint32_t a0[32], a1[32];
+                            tmem_ld_32x32b_x32(t_acc + 2 * i * kUnit, a0);
+                            tmem_ld_32x32b_x32(t_acc + (two ? 2 * i + 1 : 2 * i) * kUnit, a1);
                             tmem_wait_ld();
-                            chunk_update(best, a, sU + slot * p.u_slot_bytes, urow, half,
-                                         (u_begin + first + u) * kUnit, p, k, b_glob);
+                            box_update(best, a0, a1, two, sU + slot * p.u_slot_bytes, urow,
+                                       (u_begin + first + 2 * i) * kUnit, p, k, b_glob);
                         }
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar_u_empty + 8 * slot);
