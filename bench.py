@@ -210,6 +210,7 @@ def main():
     ap.add_argument("--workload", default="qwen3-8b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--ref-sample", type=int, default=4)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--eager", action="store_true", help="launch kernels one by one (no CUDA graph)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
 
@@ -299,6 +300,23 @@ def main():
     torch.cuda.synchronize()
     assert ds.get_error() == 0, "device error during warm-up"
 
+    # one step as a CUDA graph (launch gaps removed); eager launches if capture is refused
+    graph = None
+    if not args.eager:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step()
+            g.replay()
+            torch.cuda.synchronize()
+            assert ds.get_error() == 0
+            graph = g
+        except Exception as exc:                        # noqa: BLE001
+            print(f"# CUDA graph capture unavailable, timing eager launches: {exc}",
+                  file=sys.stderr)
+            torch.cuda.synchronize()
+    run_step = graph.replay if graph is not None else step
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.5)
@@ -311,7 +329,7 @@ def main():
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        step(ev_draft)
+        run_step()
         e1.record(stream)
         step_ev.append((e0, e1))
     torch.cuda.synchronize()
@@ -319,9 +337,15 @@ def main():
         dist.barrier()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    draft_ms = [a.elapsed_time(b) for a, b in ev_draft]
     total_ms = sum(step_ms)
     assert ds.get_error() == 0, "device error during the timed steps"
+
+    # the draft kernel alone, for its roofline (same inputs, L2 flushed before each launch)
+    for _ in range(args.steps):
+        flush.zero_()
+        step(ev_draft)
+    torch.cuda.synchronize()
+    draft_ms = [a.elapsed_time(b) for a, b in ev_draft]
 
     # ---------------- end to end through the public API with host buffers
     pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
@@ -339,7 +363,7 @@ def main():
         h.copy_(h_pin, non_blocking=True)
         anchor.copy_(anchor_pin, non_blocking=True)
         target.copy_(target_pin, non_blocking=True)
-        step()
+        run_step()
         out_x.copy_(x, non_blocking=True)
         out_L.copy_(sharding.local_lengths(Lg, rank, B) if world > 1 else Lg, non_blocking=True)
         out_acc.copy_(acc, non_blocking=True)
@@ -407,10 +431,13 @@ def main():
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": 4 * args.steps,
+            "cuda_graph": graph is not None,
             "clocks": clk,
             "draft_kernel_ms": {"mean": draft_mean, "min": min(draft_ms), "max": max(draft_ms)},
         }
         print(json.dumps(line), flush=True)
+    graph = None                                    # release the graph before the group
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
