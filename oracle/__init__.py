@@ -53,6 +53,11 @@ def _load():
         lib.oracle_schedule.restype = C.c_int
         lib.oracle_verify.argtypes = [p, p, p, C.c_int, C.c_int, p, p]
         lib.oracle_verify.restype = C.c_int
+        lib.oracle_ece.argtypes = [p, p, C.c_int, C.c_int, C.c_int]
+        lib.oracle_ece.restype = C.c_double
+        lib.oracle_sts_fit.argtypes = [p, p, C.c_int, C.c_int, C.c_double, C.c_double, C.c_int,
+                                       C.c_int, p, p, C.c_int]
+        lib.oracle_sts_fit.restype = C.c_int
         _lib = lib
     return _lib
 
@@ -160,3 +165,26 @@ def verify(x, L, target):
     if st != 0:
         raise ValueError(f"oracle_verify rejected its arguments (status {st})")
     return acc, bonus
+
+
+def ece(P, accepted, k: int, n_bins: int = 15) -> float:
+    """Expected calibration error of survival scores P [N] for position k (1-based)."""
+    P = _c(P, np.float64)
+    acc = _c(accepted, np.int32)
+    return float(_load().oracle_ece(_ptr(P), _ptr(acc), P.shape[0], int(k), int(n_bins)))
+
+
+def sts_fit(z, accepted, t_min: float = 0.5, t_step: float = 0.01, n_t: int = 451,
+            n_bins: int = 15, nthreads: int = 0):
+    """Sequential temperature scaling fit; returns (T [gamma], ece [gamma]) in fp64."""
+    z = _c(z, np.float32)
+    N, gamma = z.shape
+    acc = _c(accepted, np.int32)
+    assert acc.shape == (N,)
+    T = np.zeros(gamma)
+    e = np.zeros(gamma)
+    st = _load().oracle_sts_fit(_ptr(z), _ptr(acc), N, gamma, float(t_min), float(t_step),
+                                int(n_t), int(n_bins), _ptr(T), _ptr(e), int(nthreads))
+    if st != 0:
+        raise ValueError(f"oracle_sts_fit rejected its arguments (status {st})")
+    return T, e

@@ -362,3 +362,88 @@ int oracle_verify(const int32_t *x, const int32_t *L, const int32_t *target, int
     }
     return ORACLE_OK;
 }
+
+/* --------------------------------------------------------------------------
+ * Sequential Temperature Scaling: fitting ([G] section 5, "Sequential
+ * Temperature Scaling"): position by position, left to right, a 1-D grid
+ * search picks the temperature that minimises the expected calibration error
+ * (ECE) of the cumulative product, with the temperatures of all earlier
+ * positions already fixed.
+ *
+ * Calibration set: N blocks with raw confidence logits z[n, k-1] and accepted
+ * lengths acc[n] (number of drafts the target accepted).  Survival label at
+ * position k: y = 1 if acc[n] >= k.  For a candidate T:
+ *   P_k[n]   = P_{k-1}[n] * sigmoid(z[n, k-1] / T),   P_0 = 1
+ *   bin(p)   = min(floor(p * n_bins), n_bins - 1)     (equal-width bins on [0, 1])
+ *   ECE(T)   = sum_m |sum_{n in m} y - sum_{n in m} P_k| / N
+ * (the count-weighted mean gap |B_m|/N |mean y - mean P| written as a sum).
+ * Grid: T_i = t_min + i * t_step, i = 0 .. n_t - 1; the smallest i with the
+ * smallest ECE wins.  Outputs the chosen T per position and its ECE.
+ * ------------------------------------------------------------------------ */
+double oracle_ece(const double *P, const int32_t *acc, int N, int k, int n_bins)
+{
+    double *sy = (double *)calloc((size_t)n_bins, sizeof(double));
+    double *sp = (double *)calloc((size_t)n_bins, sizeof(double));
+    if (!sy || !sp) {
+        free(sy);
+        free(sp);
+        return -1.0;
+    }
+    for (int n = 0; n < N; ++n) {
+        int m = (int)floor(P[n] * n_bins);
+        if (m > n_bins - 1)
+            m = n_bins - 1;
+        if (m < 0)
+            m = 0;
+        sy[m] += (acc[n] >= k) ? 1.0 : 0.0;
+        sp[m] += P[n];
+    }
+    double e = 0.0;
+    for (int m = 0; m < n_bins; ++m)
+        e += fabs(sy[m] - sp[m]);
+    free(sy);
+    free(sp);
+    return e / N;
+}
+
+int oracle_sts_fit(const float *z, const int32_t *acc, int N, int gamma, double t_min,
+                   double t_step, int n_t, int n_bins, double *T_out, double *ece_out,
+                   int nthreads)
+{
+    if (N < 1 || gamma < 1 || n_t < 1 || n_bins < 1 || !(t_min > 0.0) || !(t_step >= 0.0))
+        return ORACLE_INVALID;
+    if (nthreads < 1)
+        nthreads = oracle_num_threads();
+    double *P = (double *)malloc(sizeof(double) * (size_t)N);
+    double *ece = (double *)malloc(sizeof(double) * (size_t)n_t);
+    if (!P || !ece) {
+        free(P);
+        free(ece);
+        return ORACLE_INVALID;
+    }
+    for (int n = 0; n < N; ++n)
+        P[n] = 1.0;
+    for (int k = 1; k <= gamma; ++k) {
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+        for (int i = 0; i < n_t; ++i) {
+            const double T = t_min + i * t_step;
+            double *Pk = (double *)malloc(sizeof(double) * (size_t)N);
+            for (int n = 0; n < N; ++n)
+                Pk[n] = P[n] / (1.0 + exp(-(double)z[(size_t)n * gamma + (k - 1)] / T));
+            ece[i] = oracle_ece(Pk, acc, N, k, n_bins);
+            free(Pk);
+        }
+        int best = 0;
+        for (int i = 1; i < n_t; ++i)
+            if (ece[i] < ece[best])
+                best = i;
+        const double T = t_min + best * t_step;
+        for (int n = 0; n < N; ++n)
+            P[n] = P[n] / (1.0 + exp(-(double)z[(size_t)n * gamma + (k - 1)] / T));
+        T_out[k - 1] = T;
+        ece_out[k - 1] = ece[best];
+    }
+    free(P);
+    free(ece);
+    return ORACLE_OK;
+}

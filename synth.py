@@ -30,7 +30,7 @@ import numpy as np
 
 # stream tags (one per tensor kind)
 TAG_W1, TAG_W2, TAG_U, TAG_H, TAG_ANCHOR, TAG_W, TAG_T, TAG_TARGET, TAG_ZIPF = range(1, 10)
-TAG_SCORES, TAG_VERIFY, TAG_TSTEP = 10, 11, 12
+TAG_SCORES, TAG_VERIFY, TAG_TSTEP, TAG_CALIB = 10, 11, 12, 13
 
 _THREADS = max(1, min(16, os.cpu_count() or 1))
 
@@ -325,6 +325,34 @@ def verify_inputs(B: int, gamma: int, V: int, seed: int, agree: float = 0.8):
     t = np.where(same, x, other).astype(np.int32)
     last = rng.integers(0, V, size=(B, 1)).astype(np.int32)
     return x, L, np.ascontiguousarray(np.concatenate([t, last], axis=1))
+
+
+def calibration_set(N: int, gamma: int, seed: int, q_first: float = 0.88,
+                    q_last: float = 0.78, spread: float = 2.0, scale: float = 0.6):
+    """Held-out blocks for fitting the per-position temperatures: raw confidence
+    logits z [N, gamma] (fp32) and accepted lengths [N] (int32, 0..gamma).
+
+    z[n, k] ~ N(m_k, spread^2) with m_k chosen so that the mean acceptance at
+    position k is near the linear decay q_first -> q_last.  The label process is
+    a probit link, the normal CDF Phi, so that it is not the logistic model being
+    fitted: draft k of block n is accepted with probability Phi(z[n, k] / scale) given that
+    drafts 1..k-1 were accepted, and the accepted length counts the accepted
+    drafts before the first rejection.  A small scale makes the raw logits
+    under-confident, a large one over-confident.
+    """
+    from scipy import special as _sp
+    rng = _rng(seed, TAG_CALIB, N, gamma)
+    if gamma == 1:
+        q = np.array([q_first])
+    else:
+        q = q_first + (q_last - q_first) * np.arange(gamma) / (gamma - 1)
+    # E[Phi(Z / scale)] with Z ~ N(m, spread^2) is Phi(m / sqrt(scale^2 + spread^2))
+    m = _sp.ndtri(q) * math.sqrt(scale * scale + spread * spread)
+    z = (m[None, :] + spread * rng.standard_normal((N, gamma))).astype(np.float32)
+    u = rng.random((N, gamma))
+    ok = u < _sp.ndtr(z.astype(np.float64) / scale)
+    acc = np.where(ok.all(axis=1), gamma, np.argmin(ok, axis=1)).astype(np.int32)
+    return np.ascontiguousarray(z), acc
 
 
 def draft_tokens(B: int, gamma: int, V: int, seed: int) -> np.ndarray:

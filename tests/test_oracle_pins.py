@@ -355,3 +355,108 @@ def test_verify_rejects_length_beyond_gamma(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.verify(np.zeros((1, 3), np.int32), np.array([4], np.int32),
                           np.zeros((1, 4), np.int32))
+
+
+# ---------------------------------------------------------------------------
+# Sequential Temperature Scaling, fitting (gdymind.com "DSpark", section 5,
+# "Sequential Temperature Scaling"): per position, left to right, a 1-D grid
+# search for the temperature minimising the ECE of the cumulative product, with
+# the temperatures of earlier positions frozen.
+# ---------------------------------------------------------------------------
+def test_ece_hand_computed_values(oracle_mod):
+    # one sample per bin: the ECE is the mean |y - P|
+    P = np.array([0.1, 0.2, 0.85, 0.9])
+    acc = np.array([0, 1, 1, 1], np.int32)           # labels at k = 1: acc >= 1
+    assert oracle_mod.ece(P, acc, 1) == pytest.approx((0.1 + 0.8 + 0.15 + 0.1) / 4, abs=1e-15)
+    # two samples in one bin (0.30 and 0.32 both fall in [4/15, 5/15)): the gap is
+    # taken between the bin's sums, not sample by sample
+    P = np.array([0.30, 0.32])
+    assert oracle_mod.ece(P, np.array([1, 0], np.int32), 1) == pytest.approx(abs(1 - 0.62) / 2,
+                                                                           abs=1e-15)
+    # P = 1 lands in the last bin; labels use acc >= k
+    P = np.array([1.0, 1.0, 0.0])
+    acc = np.array([3, 2, 0], np.int32)
+    assert oracle_mod.ece(P, acc, 3) == pytest.approx(1.0 / 3, abs=1e-15)
+    assert oracle_mod.ece(P, acc, 2) == pytest.approx(0.0, abs=1e-15)
+    # one bin: ECE is |mean label - mean score|
+    rng = np.random.default_rng(0)
+    P = rng.random(1000)
+    acc = rng.integers(0, 3, 1000).astype(np.int32)
+    assert oracle_mod.ece(P, acc, 1, n_bins=1) == pytest.approx(abs((acc >= 1).mean() - P.mean()),
+                                                                abs=1e-13)
+
+
+def _two_group_calibration():
+    """Two groups of 50 blocks, exactly calibrated at T = (2, 3) on the grid.
+
+    Position 1: sigmoid(z / 2) is 0.3 in group A and 0.7 in group B, and 15 and 35
+    blocks of them accept.  Position 2: sigmoid(z / 3) is 0.8 for every block,
+    so the cumulative products are 0.24 and 0.56, and 12 and 28 blocks accept
+    both drafts.  Every other temperature moves the scores off the label rates.
+    """
+    za = 2.0 * math.log(0.3 / 0.7)
+    zb = 2.0 * math.log(0.7 / 0.3)
+    z2 = 3.0 * math.log(4.0)
+    z = np.zeros((100, 2), np.float32)
+    z[:50, 0], z[50:, 0], z[:, 1] = za, zb, z2
+    acc = np.zeros(100, np.int32)
+    acc[:12] = 2; acc[12:15] = 1                       # group A: 15 accept #1, 12 accept #2
+    acc[50:78] = 2; acc[78:85] = 1                     # group B: 35 accept #1, 28 accept #2
+    return z, acc
+
+
+def test_sts_fit_exact_calibration_is_found(oracle_mod):
+    z, acc = _two_group_calibration()
+    T, e = oracle_mod.sts_fit(z, acc, t_min=0.5, t_step=0.01, n_t=451)
+    # z is stored in fp32, so the zero of the ECE sits within 1e-6 of (2, 3)
+    np.testing.assert_allclose(T, [2.0, 3.0], atol=1e-9)
+    assert (e < 1e-6).all()
+    # with position 1 frozen at its raw scores (T = 1: 0.155 and 0.845) instead of
+    # its fitted ones, the product at T_2 = 3 would be 0.124 and 0.676 against
+    # label rates 0.24 and 0.56, so the zero at (2, 3) pins the frozen prefix too
+
+
+def test_sts_fit_scales_with_the_logits(oracle_mod):
+    # sigmoid((2 z) / (2 T)) = sigmoid(z / T) bit for bit, and the doubled grid
+    # 1.0 + 0.02 i is exactly twice 0.5 + 0.01 i: the fit must double exactly
+    z, acc = synth.calibration_set(3000, 6, seed=3)
+    T, e = oracle_mod.sts_fit(z, acc, t_min=0.5, t_step=0.01, n_t=451)
+    T2, e2 = oracle_mod.sts_fit(2 * z, acc, t_min=1.0, t_step=0.02, n_t=451)
+    np.testing.assert_array_equal(T2, 2 * T)
+    np.testing.assert_array_equal(e2, e)
+
+
+def test_sts_fit_each_choice_is_the_grid_minimum(oracle_mod):
+    # with T_1..T_{k-1} frozen at the fit, no grid temperature at k beats T_k;
+    # the ECE of each candidate is the oracle's own ECE of the explicit product
+    z, acc = synth.calibration_set(800, 4, seed=4)
+    grid = 0.5 + 0.01 * np.arange(451)
+    T, e = oracle_mod.sts_fit(z, acc)
+    P = np.ones(800)
+    for k in range(4):
+        eces = [oracle_mod.ece(P * special.expit(z[:, k].astype(np.float64) / t), acc, k + 1)
+                for t in grid]
+        i = int(np.argmin(eces))
+        assert T[k] == grid[i] and e[k] == pytest.approx(eces[i], abs=1e-15)
+        P = P * special.expit(z[:, k].astype(np.float64) / T[k])
+
+
+def test_sts_fit_recovers_the_true_temperature(oracle_mod):
+    # labels drawn from an exactly logistic survival chain with known T*: the
+    # fitted temperatures converge to T* as the calibration set grows
+    rng = np.random.default_rng(7)
+    N, Tstar = 60000, np.array([1.5, 2.4, 3.3])
+    z = rng.normal(2.5, 2.5, (N, 3)).astype(np.float32)
+    ok = rng.random((N, 3)) < special.expit(z.astype(np.float64) / Tstar)
+    acc = np.where(ok.all(axis=1), 3, np.argmin(ok, axis=1)).astype(np.int32)
+    T, e = oracle_mod.sts_fit(z, acc)
+    np.testing.assert_allclose(T, Tstar, atol=0.2)
+    assert (e < 0.01).all()
+
+
+def test_sts_fit_rejects_bad_arguments(oracle_mod):
+    z, acc = _two_group_calibration()
+    with pytest.raises(ValueError):
+        oracle_mod.sts_fit(z, acc, t_min=0.0)
+    with pytest.raises(ValueError):
+        oracle_mod.sts_fit(z, acc, n_bins=0)
