@@ -427,6 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tile_span(t, n_units, ntiles, first, count);
                         const int v0 = (u_begin + first) * kUnit;
                         const int nbox = (count + 1) >> 1;          // 64-column boxes
+                        if (mt == 0 && t == 0) DSPARK_TRACE_AT(k, 7);
+                        if (mt == num_mt - 1 && t == ntiles - 1) DSPARK_TRACE_AT(k, 8);
                         for (int ks = 0; ks < kKSlices; ++ks) {
                             if (!wait_phase(bar_w2_empty + 8 * w2.slot, w2.phase ^ 1u, ctl, p)) {
                                 ok = false;
@@ -466,9 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 break;
                             }
                             const uint32_t bar = bar_u_full + 8 * ur.slot;
+                            if (mt == 0 && t == 0 && u == 0) DSPARK_TRACE_AT(k, 11);
+                            if (mt == num_mt - 1 && t == ntiles - 1 && u + 2 >= count) DSPARK_TRACE_AT(k, 12);
                             mbar_arrive_expect_tx(bar, u_tx);
                             tma_load_3d(sU + ur.slot * p.u_slot_bytes, &tm_u, bar, v0 + u * kUnit,
                                         k - 1, mt * M, pol_u);
+
                             ++issued;
                             ur.next(p.u_slots);
                         }
@@ -498,17 +503,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tile_span(t, n_units, ntiles, first, count);
                         const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(M),
                                                               static_cast<uint32_t>(count * kUnit), 1);
+#ifdef DSPARK_TRACE
+                        const uint64_t tw0 = globaltimer_ns();
+#endif
                         if (!wait_phase(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p)) {
                             ok = false;
                             break;
                         }
+                        DSPARK_TRACE_ADD(k, 14, globaltimer_ns() - tw0);
                         tc_fence_after();
                         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
                         for (int ks = 0; ks < kKSlices; ++ks) {
+#ifdef DSPARK_TRACE
+                            const uint64_t tw1 = globaltimer_ns();
+#endif
                             if (!wait_phase(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
                                 ok = false;
                                 break;
                             }
+                            DSPARK_TRACE_ADD(k, 13, globaltimer_ns() - tw1);
                             tc_fence_after();
                             // descriptors differ only in the start-address field (bits 0..13,
                             // 16-byte units): advance them with plain adds
@@ -527,6 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (!ok) break;
                         if (!ok) break;
+                        if (mt == 0 && t == 0) DSPARK_TRACE_AT(k, 9);
+                        if (mt == num_mt - 1 && t == ntiles - 1) DSPARK_TRACE_AT(k, 10);
                         umma_commit(bar_tfull + 8 * acc.slot);
                         acc.next(kAcc);
                     }
@@ -563,32 +578,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             next_tok[mt] = (lane_row && b < p.B) ? checked_token(p.anchor[b], p.V) : -1;
         }
 
+        // gather A = W1[x_{k-1}] of M tile gmt (K-major, 128-byte swizzle), all rows in
+        // flight; the MMA must have released A (aempty) before this is called
+        auto gather = [&](int gmt) {
+            const int my_tok = next_tok[gmt];
+            for (int i = 0; i < gather_rows; ++i) {
+                const int src_lane = half * gather_rows + i;
+                const int tok = __shfl_sync(0xFFFFFFFFu, my_tok, src_lane);
+                const int r = q * rq + src_lane;
+                const uint32_t dst = sA + chunk * a_chunk + r * 128 + ((unit ^ (r & 7)) << 4);
+                if (tok >= 0)
+                    cp_async_16(dst, p.W1 + static_cast<size_t>(tok) * kRank + lane * 8);
+                else
+                    sts128_zero(dst);
+            }
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_afull);
+            ++mt_count;
+        };
+
         for (int k = 1; k <= p.gamma && ok; ++k) {
+            if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
+                ok = false;
+                break;
+            }
+            if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 0);
+            gather(0);
+            if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 1);
             for (int mt = 0; mt < num_mt && ok; ++mt) {
                 const int m0 = mt * M;
                 const int my_b = m0 + row;
-                // ---- gather A = W1[x_{k-1}] (K-major, 128-byte swizzle), all rows in flight
-                if (!__all_sync(0xFFFFFFFFu,
-                                wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
-                    ok = false;
-                    break;
-                }
-                const int my_tok = next_tok[mt];
-                for (int i = 0; i < gather_rows; ++i) {
-                    const int src_lane = half * gather_rows + i;
-                    const int tok = __shfl_sync(0xFFFFFFFFu, my_tok, src_lane);
-                    const int r = q * rq + src_lane;
-                    const uint32_t dst = sA + chunk * a_chunk + r * 128 + ((unit ^ (r & 7)) << 4);
-                    if (tok >= 0)
-                        cp_async_16(dst, p.W1 + static_cast<size_t>(tok) * kRank + lane * 8);
-                    else
-                        sts128_zero(dst);
-                }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_afull);
-                ++mt_count;
+                // the next M tile's rows are gathered as soon as the MMA has released A, so
+                // the tensor core does not wait for this tile's epilogue to finish
+                bool next_gathered = mt + 1 >= num_mt;
 
                 // ---- vocabulary tiles of this CTA: this warp takes chunks u with u % 2 == half
                 const bool active = (m0 + q * rq) < p.B;
@@ -604,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
+                    if (threadIdx.x == 0 && mt == 0 && t == 0) DSPARK_TRACE_AT(k, 2);
                     // box i of the tile holds chunks 2i and 2i + 1; this warp takes boxes i = half,
                     // half + 2, ... and reduces both chunks of a box together
                     const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
@@ -612,10 +637,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const long long pos = u_pos + i;
                         const int slot = static_cast<int>(pos % p.u_slots);
                         const uint32_t par = static_cast<uint32_t>((pos / p.u_slots) & 1);
+#ifdef DSPARK_TRACE
+                        const uint64_t tw2 = globaltimer_ns();
+#endif
                         if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_u_full + 8 * slot, par, ctl, p))) {
                             ok = false;
                             break;
                         }
+                        if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 15, globaltimer_ns() - tw2);
                         if (active) {
                             const bool two = 2 * i + 1 < count;
                             uint32_t a0[32], a1[32];
@@ -634,8 +663,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar_tempty + 8 * acc.slot);
                     acc.next(kAcc);
+                    if (!next_gathered &&
+                        __all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty, (mt_count & 1u) ^ 1u))) {
+                        gather(mt + 1);
+                        next_gathered = true;
+                    }
                 }
                 if (!ok) break;
+                if (!next_gathered) {
+                    if (!__all_sync(0xFFFFFFFFu,
+                                    wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
+                        ok = false;
+                        break;
+                    }
+                    gather(mt + 1);
+                }
                 if (lane_row && my_b < p.B) {
                     const unsigned long long key = argmax_key(best.s, best.v);
                     atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + my_b], key);
@@ -645,9 +687,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
 
             // ---- grid barrier: every CTA has combined its rows of position k
+            if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 3);
             epi_sync();
             if (threadIdx.x == 0 && ok && !*reinterpret_cast<volatile int *>(&ctl.abort)) {
                 red_release_add_u32(p.barrier, 1u);
+                DSPARK_TRACE_AT(k, 4);
                 const uint32_t target = static_cast<uint32_t>(k) * static_cast<uint32_t>(G) +
                                         static_cast<uint32_t>(p.barrier_extra);
                 const uint64_t t0 = globaltimer_ns();
@@ -661,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                 }
+                DSPARK_TRACE_AT(k, 5);
             }
             epi_sync();
             if (!ok || *reinterpret_cast<volatile int *>(&ctl.abort)) {
@@ -680,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     p.logit_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = my_logit[mt];
                 }
             }
+            if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 6);
         }
     }
 
