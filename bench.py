@@ -9,6 +9,7 @@ second, B * gamma / step time, summed over ranks.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload qwen3-8b]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+    python bench.py --stage sts-fit        # fitting the STS temperatures (offline calibration)
 
 With N > 1 (torchrun, one process per GPU) every rank drafts its own B requests
 (weak scaling) and the survival scores of all ranks are all-gathered over NCCL
@@ -201,6 +202,92 @@ def cpu_baseline(wl, inp, target, budget_s):
                                         f"(draft, confidence, schedule, verify), {total:.1f} s"}
 
 
+STS_METRIC = "STS fit candidate evaluations/s (blocks x gamma x grid temperatures)"
+STS_UNIT = "evaluations/s"
+
+
+def run_sts_fit(args):
+    """Time dspark_sts_fit on the held-out calibration set (65536 blocks, gamma = 16,
+    451 temperatures 0.5..5.0, 15 bins); the oracle's fit on a subset is the CPU baseline."""
+    import torch
+    import speculative_decoding_drafter_head_b200 as ds
+
+    N, gamma = synth.STS_CALIBRATION_N, synth.STS_CALIBRATION_GAMMA
+    n_t, n_bins = 451, 15
+    z_h, acc_h = synth.calibration_set(N, gamma, 0)
+    z, acc = torch.from_numpy(z_h).cuda(), torch.from_numpy(acc_h).cuda()
+    ws = torch.empty(ds.sts_fit_workspace_bytes(N, gamma, n_t, n_bins), dtype=torch.uint8,
+                     device="cuda")
+    idx = torch.empty(gamma, dtype=torch.int32, device="cuda")
+    T = torch.empty(gamma, dtype=torch.float32, device="cuda")
+    e = torch.empty(gamma, dtype=torch.float64, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        ds.sts_fit(z, acc, idx, T, e, ws)
+    torch.cuda.synchronize()
+    assert ds.get_error() == 0
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.5)
+    evs = []
+    for _ in range(args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ds.sts_fit(z, acc, idx, T, e, ws)
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    evals = float(N) * gamma * n_t
+    value = evals * args.steps / (sum(ms) / 1e3)
+
+    # e2e: calibration set copied from pinned host memory, temperatures read back
+    z_pin, acc_pin = torch.from_numpy(z_h).pin_memory(), torch.from_numpy(acc_h).pin_memory()
+    T_pin = torch.empty(gamma, dtype=torch.float32).pin_memory()
+    e2e = []
+    for it in range(args.steps + 1):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        z.copy_(z_pin, non_blocking=True)
+        acc.copy_(acc_pin, non_blocking=True)
+        ds.sts_fit(z, acc, idx, T, e, ws)
+        T_pin.copy_(T, non_blocking=True)
+        e1.record(stream)
+        if it:
+            e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e)
+
+    import oracle
+    oracle.build()
+    n_cpu = 4096
+    t0 = time.perf_counter()
+    oracle.sts_fit(z_h[:n_cpu], acc_h[:n_cpu], n_t=n_t, n_bins=n_bins)
+    cpu_s = time.perf_counter() - t0
+    line = {
+        "metric": STS_METRIC, "value": value, "unit": STS_UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": statistics.mean(ms), "higher_is_better": True,
+        "scaling": "none", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"sts-calibration N={N} gamma={gamma} n_t={n_t} bins={n_bins}",
+                   "l2_flush": False, "inputs_bytes": int(z_h.nbytes + acc_h.nbytes)},
+        "roofline": {"bound": "alu", "kernel": "sts_hist_kernel",
+                     "note": "fp64 exp/divide per candidate; fp64 pipe share from ncu"},
+        "cpu_baseline": {"value": n_cpu * gamma * n_t / cpu_s, "unit": STS_UNIT,
+                         "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"oracle fit of the first {n_cpu} of {N} blocks"},
+        "e2e": {"value": evals * args.steps / (e2e_ms / 1e3), "unit": STS_UNIT,
+                "h2d_bytes_per_step": int(z_h.nbytes + acc_h.nbytes),
+                "d2h_bytes_per_step": gamma * 4},
+        "gpu_launches": (2 * gamma) * args.steps,
+        "clocks": clk,
+        "T": [round(float(v), 2) for v in T.cpu()],
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -211,8 +298,14 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=4)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--eager", action="store_true", help="launch kernels one by one (no CUDA graph)")
+    ap.add_argument("--stage", default="path", choices=["path", "sts-fit"],
+                    help="path: the per-step hot path; sts-fit: the temperature fit")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
+    if args.stage == "sts-fit":
+        if int(os.environ.get("RANK", "0")) == 0 and args.impl == "ours":
+            run_sts_fit(args)
+        return
 
     if args.impl == "reference":
         run_reference(args, wl)

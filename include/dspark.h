@@ -153,6 +153,44 @@ int dspark_verify_prefix(const int32_t *x, const int32_t *L, const int32_t *targ
                          dspark_stream_t stream);
 
 /*
+ * Sequential Temperature Scaling: fitting the per-position temperatures T [gamma]
+ * that dspark_confidence_sts divides the confidence logits by.
+ * [G] section 5 "Sequential Temperature Scaling": the joint (survival) probability is
+ * calibrated position by position from left to right; at each position a 1-D grid
+ * search picks the temperature minimising the expected calibration error (ECE) of the
+ * cumulative product, with the temperatures of earlier positions kept fixed.
+ *
+ * Calibration set: N held-out draft blocks with raw confidence logits z[n, k-1] (the
+ * logit before temperature scaling) and accepted lengths accepted[n] in 0..gamma.
+ * For k = 1..gamma, label y = (accepted[n] >= k) and for each candidate
+ * T_i = t_min + i t_step, i = 0..n_t-1:
+ *   p_i[n] = P_{k-1}[n] / (1 + exp(-z[n, k-1] / T_i))      (fp64; P_0 = 1)
+ *   ECE_i  = sum over bins m of |sum_{n in m} y - sum_{n in m} p_i| / N,
+ *            bin(p) = min(floor(p n_bins), n_bins - 1)       (equal-width bins on [0, 1])
+ * index_out[k-1] = the smallest i with the smallest ECE_i; T_out[k-1] = T_i (fp32);
+ * ece_out[k-1] = ECE_i; then P_k = P_{k-1} / (1 + exp(-z[., k-1] / T_i)).
+ * p is formed as P / (1 + exp(-z (1/T))) with a Newton-refined reciprocal (a
+ * few ulp from the fp64 quotient).  Each CTA's fp64 bin sums are rounded to 2^-40 fixed
+ * point before they are added across CTAs, so the result does not depend on the order
+ * in which CTAs finish (an ECE moves by at most (CTAs x bins) 2^-41 / N); ties are
+ * decided on those exact integer sums.
+ *
+ *   z          [N, gamma] fp32
+ *   accepted   [N] int32
+ *   index_out  [gamma] int32   (device memory; also read by the later positions)
+ *   T_out      [gamma] fp32,  ece_out [gamma] fp64
+ *   workspace, workspace_bytes >= dspark_sts_fit_workspace_bytes(N, gamma, n_t, n_bins)
+ * Supported sizes: 1 <= N < 2^23, 1 <= gamma <= 64, 1 <= n_t <= 2^20,
+ * 1 <= n_bins <= 256; t_min > 0, t_step >= 0.  Errors: DSPARK_INVALID_ARG (null or
+ * misaligned pointer, bad grid), DSPARK_UNSUPPORTED_SHAPE, DSPARK_WORKSPACE_TOO_SMALL.
+ */
+size_t dspark_sts_fit_workspace_bytes(int N, int gamma, int n_t, int n_bins);
+int dspark_sts_fit(const float *z, const int32_t *accepted, int N, int gamma, double t_min,
+                   double t_step, int n_t, int n_bins, int32_t *index_out, float *T_out,
+                   double *ece_out, void *workspace, size_t workspace_bytes,
+                   dspark_stream_t stream);
+
+/*
  * The prefix scheduler for callers that cannot allocate device memory.
  * (No counterpart on the DSpark pages: this is an interface convenience.)
  *

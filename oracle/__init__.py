@@ -56,7 +56,7 @@ def _load():
         lib.oracle_ece.argtypes = [p, p, C.c_int, C.c_int, C.c_int]
         lib.oracle_ece.restype = C.c_double
         lib.oracle_sts_fit.argtypes = [p, p, C.c_int, C.c_int, C.c_double, C.c_double, C.c_int,
-                                       C.c_int, p, p, C.c_int]
+                                       C.c_int, p, p, p, p, C.c_int]
         lib.oracle_sts_fit.restype = C.c_int
         _lib = lib
     return _lib
@@ -175,16 +175,26 @@ def ece(P, accepted, k: int, n_bins: int = 15) -> float:
 
 
 def sts_fit(z, accepted, t_min: float = 0.5, t_step: float = 0.01, n_t: int = 451,
-            n_bins: int = 15, nthreads: int = 0):
-    """Sequential temperature scaling fit; returns (T [gamma], ece [gamma]) in fp64."""
+            n_bins: int = 15, T_fixed=None, return_grid: bool = False, nthreads: int = 0):
+    """Sequential temperature scaling fit; returns (T [gamma], ece [gamma]) in fp64.
+
+    With T_fixed [gamma], each position is frozen at T_fixed[k] rather than at its
+    own choice before the next position is fitted.  With return_grid, a third
+    value holds every candidate's ECE [gamma, n_t].
+    """
     z = _c(z, np.float32)
     N, gamma = z.shape
     acc = _c(accepted, np.int32)
     assert acc.shape == (N,)
+    fixed = None if T_fixed is None else _c(T_fixed, np.float64)
+    assert fixed is None or fixed.shape == (gamma,)
     T = np.zeros(gamma)
     e = np.zeros(gamma)
+    grid = np.zeros((gamma, n_t)) if return_grid else None
     st = _load().oracle_sts_fit(_ptr(z), _ptr(acc), N, gamma, float(t_min), float(t_step),
-                                int(n_t), int(n_bins), _ptr(T), _ptr(e), int(nthreads))
+                                int(n_t), int(n_bins), None if fixed is None else _ptr(fixed),
+                                _ptr(T), _ptr(e), None if grid is None else _ptr(grid),
+                                int(nthreads))
     if st != 0:
         raise ValueError(f"oracle_sts_fit rejected its arguments (status {st})")
-    return T, e
+    return (T, e, grid) if return_grid else (T, e)

@@ -378,7 +378,10 @@ int oracle_verify(const int32_t *x, const int32_t *L, const int32_t *target, int
  *   ECE(T)   = sum_m |sum_{n in m} y - sum_{n in m} P_k| / N
  * (the count-weighted mean gap |B_m|/N |mean y - mean P| written as a sum).
  * Grid: T_i = t_min + i * t_step, i = 0 .. n_t - 1; the smallest i with the
- * smallest ECE wins.  Outputs the chosen T per position and its ECE.
+ * smallest ECE wins.  Outputs the chosen T per position and its ECE, and, when
+ * ece_grid is given, every candidate's ECE [gamma][n_t].  When T_fixed is given,
+ * position k is frozen at T_fixed[k-1] instead of the chosen T (so that another
+ * implementation's choices can be scored), while T_out still reports the choice.
  * ------------------------------------------------------------------------ */
 double oracle_ece(const double *P, const int32_t *acc, int N, int k, int n_bins)
 {
@@ -407,8 +410,8 @@ double oracle_ece(const double *P, const int32_t *acc, int N, int k, int n_bins)
 }
 
 int oracle_sts_fit(const float *z, const int32_t *acc, int N, int gamma, double t_min,
-                   double t_step, int n_t, int n_bins, double *T_out, double *ece_out,
-                   int nthreads)
+                   double t_step, int n_t, int n_bins, const double *T_fixed, double *T_out,
+                   double *ece_out, double *ece_grid, int nthreads)
 {
     if (N < 1 || gamma < 1 || n_t < 1 || n_bins < 1 || !(t_min > 0.0) || !(t_step >= 0.0))
         return ORACLE_INVALID;
@@ -437,11 +440,14 @@ int oracle_sts_fit(const float *z, const int32_t *acc, int N, int gamma, double 
         for (int i = 1; i < n_t; ++i)
             if (ece[i] < ece[best])
                 best = i;
-        const double T = t_min + best * t_step;
+        if (ece_grid)
+            for (int i = 0; i < n_t; ++i)
+                ece_grid[(size_t)(k - 1) * n_t + i] = ece[i];
+        T_out[k - 1] = t_min + best * t_step;
+        ece_out[k - 1] = ece[best];
+        const double T = T_fixed ? T_fixed[k - 1] : T_out[k - 1];
         for (int n = 0; n < N; ++n)
             P[n] = P[n] / (1.0 + exp(-(double)z[(size_t)n * gamma + (k - 1)] / T));
-        T_out[k - 1] = T;
-        ece_out[k - 1] = ece[best];
     }
     free(P);
     free(ece);

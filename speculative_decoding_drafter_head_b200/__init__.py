@@ -10,6 +10,7 @@ raises.
     confidence_sts    confidence head, sequential temperature scaling, survival product
     schedule_prefix   hardware-aware prefix scheduler (global top-N + scan)
     verify_prefix     strict prefix-match verification
+    sts_fit           fitting the per-position temperatures (ECE grid search)
 """
 from __future__ import annotations
 
@@ -20,7 +21,7 @@ from . import _build
 
 __all__ = [
     "DSparkError", "load", "workspace_bytes", "draft_step", "confidence_sts", "schedule_prefix",
-    "verify_prefix", "get_error", "status_string", "set_wait_timeout_ns", "debug_barrier_extra",
+    "verify_prefix", "sts_fit_workspace_bytes", "sts_fit", "get_error", "status_string", "set_wait_timeout_ns", "debug_barrier_extra",
     "STATUS",
 ]
 
@@ -33,6 +34,7 @@ EXPORTED = (
     "dspark_status_string", "dspark_workspace_bytes", "dspark_draft_step",
     "dspark_confidence_sts", "dspark_schedule_prefix", "dspark_verify_prefix",
     "dspark_get_error", "dspark_set_wait_timeout_ns", "dspark_debug_barrier_extra",
+    "dspark_sts_fit_workspace_bytes", "dspark_sts_fit",
 )
 
 _lib = None
@@ -63,11 +65,15 @@ def load(build_if_missing: bool = True):
     lib.dspark_confidence_sts.argtypes = [p, p, p, p, p, f32, p, i, i, i, i, i, p, p, p]
     lib.dspark_schedule_prefix.argtypes = [p, i, i, p, p, p, p, p, sz, p]
     lib.dspark_verify_prefix.argtypes = [p, p, p, i, i, p, p, p]
+    lib.dspark_sts_fit_workspace_bytes.argtypes = [i, i, i, i]
+    lib.dspark_sts_fit_workspace_bytes.restype = sz
+    lib.dspark_sts_fit.argtypes = [p, p, i, i, C.c_double, C.c_double, i, i, p, p, p, p, sz, p]
     lib.dspark_get_error.argtypes = [p, C.POINTER(C.c_int)]
     lib.dspark_set_wait_timeout_ns.argtypes = [u64]
     lib.dspark_debug_barrier_extra.argtypes = [i]
     for name in EXPORTED:
-        if name != "dspark_status_string" and name != "dspark_workspace_bytes":
+        if name not in ("dspark_status_string", "dspark_workspace_bytes",
+                        "dspark_sts_fit_workspace_bytes"):
             getattr(lib, name).restype = i
     _lib = lib
     return lib
@@ -153,6 +159,24 @@ def verify_prefix(x, L, target, accepted_out, bonus_out, stream=None):
         B, gamma, _dev(accepted_out, torch.int32, "accepted_out"),
         _dev(bonus_out, torch.int32, "bonus_out"), _stream(stream))
     _check("dspark_verify_prefix", st)
+
+
+def sts_fit_workspace_bytes(N: int, gamma: int, n_t: int, n_bins: int) -> int:
+    return int(load().dspark_sts_fit_workspace_bytes(N, gamma, n_t, n_bins))
+
+
+def sts_fit(z, accepted, index_out, T_out, ece_out, workspace, t_min: float = 0.5,
+            t_step: float = 0.01, n_t: int = 451, n_bins: int = 15, stream=None):
+    """Fit the per-position STS temperatures on a calibration set (see dspark_sts_fit)."""
+    import torch
+    N, gamma = z.shape
+    st = load().dspark_sts_fit(
+        _dev(z, torch.float32, "z"), _dev(accepted, torch.int32, "accepted"), N, gamma,
+        float(t_min), float(t_step), int(n_t), int(n_bins),
+        _dev(index_out, torch.int32, "index_out"), _dev(T_out, torch.float32, "T_out"),
+        _dev(ece_out, torch.float64, "ece_out"), _dev(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream))
+    _check("dspark_sts_fit", st)
 
 
 def get_error(stream=None) -> int:

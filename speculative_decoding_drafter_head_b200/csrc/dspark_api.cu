@@ -14,6 +14,7 @@
 #include "markov_draft.cuh"
 #include "ptx.cuh"
 #include "schedule_prefix.cuh"
+#include "sts_fit.cuh"
 #include "verify_prefix.cuh"
 
 namespace {
@@ -88,6 +89,19 @@ size_t sched_ws(int n)
 }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_CUDA_ERROR; }
+
+// STS-fit workspace: frozen products [2][N] f64, then label counts [gamma][n_t][n_bins]
+// u32, then fixed-point sums [gamma][n_t][n_bins] u64.
+struct StsFitLayout {
+    size_t p_bytes, cnt_bytes, sq_bytes;
+    size_t total() const { return p_bytes + cnt_bytes + sq_bytes; }
+};
+
+StsFitLayout sts_fit_layout(int N, int gamma, int n_t, int n_bins)
+{
+    const size_t cells = static_cast<size_t>(gamma) * n_t * n_bins;
+    return {round_up(static_cast<size_t>(N) * 16, 256), round_up(cells * 4, 256), cells * 8};
+}
 
 }  // namespace
 
@@ -313,6 +327,79 @@ int dspark_verify_prefix(const int32_t *x, const int32_t *L, const int32_t *targ
     return from_cuda(cudaGetLastError());
 }
 
+size_t dspark_sts_fit_workspace_bytes(int N, int gamma, int n_t, int n_bins)
+{
+    if (N < 1 || gamma < 1 || n_t < 1 || n_bins < 1) return 0;
+    return sts_fit_layout(N, gamma, n_t, n_bins).total();
+}
+
+int dspark_sts_fit(const float *z, const int32_t *accepted, int N, int gamma, double t_min,
+                   double t_step, int n_t, int n_bins, int32_t *index_out, float *T_out,
+                   double *ece_out, void *workspace, size_t workspace_bytes,
+                   dspark_stream_t stream)
+{
+    namespace F = dspark::stsfit;
+    if (!z || !accepted || !index_out || !T_out || !ece_out || !workspace)
+        return DSPARK_INVALID_ARG;
+    if (!aligned(z, 4) || !aligned(accepted, 4) || !aligned(index_out, 4) || !aligned(T_out, 4) ||
+        !aligned(ece_out, 8) || !aligned(workspace, 256))
+        return DSPARK_INVALID_ARG;
+    const double t_max = t_min + static_cast<double>(n_t - 1) * t_step;
+    if (!(t_min > 0.0) || !(t_step >= 0.0) || !(t_max < 1e300)) return DSPARK_INVALID_ARG;
+    if (N < 1 || N > F::kMaxN || gamma < 1 || gamma > 64 || n_t < 1 || n_t > (1 << 20) ||
+        n_bins < 1 || n_bins > F::kMaxBins)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    const StsFitLayout lay = sts_fit_layout(N, gamma, n_t, n_bins);
+    if (workspace_bytes < lay.total()) return DSPARK_WORKSPACE_TOO_SMALL;
+    DeviceInfo *dev = nullptr;
+    if (int st = current_device(&dev)) return st;
+
+    int tpb = static_cast<int>(round_up(static_cast<size_t>(n_t), 32));
+    if (tpb > F::kMaxThreads) tpb = F::kMaxThreads;
+    while (F::hist_smem_bytes(tpb, n_bins) > 200 * 1024 && tpb > 32)
+        tpb = static_cast<int>(round_up(static_cast<size_t>(tpb / 2), 32));
+    const size_t smem = F::hist_smem_bytes(tpb, n_bins);
+    const int gy = (n_t + tpb - 1) / tpb;
+    if (gy > 65535) return DSPARK_UNSUPPORTED_SHAPE;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(F::sts_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DSPARK_CUDA_ERROR;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, F::sts_hist_kernel, tpb, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        return DSPARK_CUDA_ERROR;
+    int gx = per_sm * dev->sms / gy;             // one even share of the samples per CTA slot
+    if (gx > (N + 63) / 64) gx = (N + 63) / 64;  // but no share below 64 samples
+    if (gx < 1) gx = 1;
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    F::Params prm;
+    prm.z = z;
+    prm.acc = accepted;
+    prm.N = N;
+    prm.gamma = gamma;
+    prm.t_min = t_min;
+    prm.t_step = t_step;
+    prm.n_t = n_t;
+    prm.n_bins = n_bins;
+    prm.P = reinterpret_cast<double *>(ws);
+    prm.idx = index_out;
+    prm.T_out = T_out;
+    prm.ece_out = ece_out;
+    prm.cnt = reinterpret_cast<unsigned int *>(ws + lay.p_bytes);
+    prm.sq = reinterpret_cast<unsigned long long *>(ws + lay.p_bytes + lay.cnt_bytes);
+    if (cudaMemsetAsync(ws + lay.p_bytes, 0, lay.cnt_bytes + lay.sq_bytes, stream) != cudaSuccess)
+        return DSPARK_CUDA_ERROR;
+    for (int k = 1; k <= gamma; ++k) {
+        prm.k = k;
+        F::sts_hist_kernel<<<dim3(gx, gy), tpb, smem, stream>>>(prm);
+        F::sts_pick_kernel<<<1, F::kPickThreads, 0, stream>>>(prm);
+    }
+    return from_cuda(cudaGetLastError());
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------
@@ -407,3 +494,12 @@ int dspark_get_error(dspark_stream_t stream, int *status)
 }
 
 }  // extern "C"
+
+#ifdef DSPARK_TRACE
+// Trace builds only: copy the draft kernel's timeline (see DSPARK_TRACE_AT).
+extern "C" int dspark_trace_copy(void *host, size_t bytes)
+{
+    return cudaMemcpyFromSymbol(host, dspark::g_trace, bytes) == cudaSuccess ? DSPARK_OK
+                                                                              : DSPARK_CUDA_ERROR;
+}
+#endif

@@ -327,8 +327,13 @@ def verify_inputs(B: int, gamma: int, V: int, seed: int, agree: float = 0.8):
     return x, L, np.ascontiguousarray(np.concatenate([t, last], axis=1))
 
 
+# held-out calibration set for fitting the temperatures: 65536 blocks of gamma = 16
+STS_CALIBRATION_N = 65536
+STS_CALIBRATION_GAMMA = 16
+
+
 def calibration_set(N: int, gamma: int, seed: int, q_first: float = 0.88,
-                    q_last: float = 0.78, spread: float = 2.0, scale: float = 0.6):
+                    q_last: float = 0.78, spread: float = 2.0, scale: float = 3.4):
     """Held-out blocks for fitting the per-position temperatures: raw confidence
     logits z [N, gamma] (fp32) and accepted lengths [N] (int32, 0..gamma).
 
@@ -338,7 +343,8 @@ def calibration_set(N: int, gamma: int, seed: int, q_first: float = 0.88,
     fitted: draft k of block n is accepted with probability Phi(z[n, k] / scale) given that
     drafts 1..k-1 were accepted, and the accepted length counts the accepted
     drafts before the first rejection.  A small scale makes the raw logits
-    under-confident, a large one over-confident.
+    under-confident, a large one over-confident; the default 3.4 puts the fitted
+    temperatures near 2 (the logistic and normal CDFs match at a factor of ~1.7).
     """
     from scipy import special as _sp
     rng = _rng(seed, TAG_CALIB, N, gamma)

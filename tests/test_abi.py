@@ -90,3 +90,26 @@ def test_binding_rejects_cpu_tensors():
         ds.verify_prefix(torch.zeros(2, 3, dtype=torch.int32), torch.zeros(2, dtype=torch.int32),
                          torch.zeros(2, 4, dtype=torch.int32), torch.zeros(2, dtype=torch.int32),
                          torch.zeros(2, dtype=torch.int32))
+
+
+def test_sts_fit_host_checks():
+    lib = ds.load()
+    f = lib.dspark_sts_fit
+    need = ds.sts_fit_workspace_bytes(4096, 16, 451, 15)
+    assert need >= 4096 * 16 + 16 * 451 * 15 * 12
+    assert ds.sts_fit_workspace_bytes(0, 16, 451, 15) == 0
+    args = dict(z=_FAKE, acc=_FAKE, N=4096, gamma=16, t_min=0.5, t_step=0.01, n_t=451, n_bins=15,
+                idx=_FAKE, T=_FAKE, e=_FAKE, ws=C.c_void_p(0x10000), wsb=need, stream=None)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return f(a["z"], a["acc"], a["N"], a["gamma"], a["t_min"], a["t_step"], a["n_t"],
+                 a["n_bins"], a["idx"], a["T"], a["e"], a["ws"], a["wsb"], a["stream"])
+
+    assert call(z=None) == 1
+    assert call(e=C.c_void_p(0x10004)) == 1            # fp64 output not 8-byte aligned
+    assert call(ws=C.c_void_p(0x10080)) == 1           # workspace not 256-byte aligned
+    assert call(t_min=0.0) == 1 and call(t_step=-0.01) == 1
+    assert call(N=0) == 2 and call(N=1 << 23) == 2     # fixed-point sums need N < 2^23
+    assert call(gamma=65) == 2 and call(n_bins=257) == 2 and call(n_t=0) == 2
+    assert call(wsb=need - 1) == 3

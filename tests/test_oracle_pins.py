@@ -427,18 +427,25 @@ def test_sts_fit_scales_with_the_logits(oracle_mod):
 
 
 def test_sts_fit_each_choice_is_the_grid_minimum(oracle_mod):
-    # with T_1..T_{k-1} frozen at the fit, no grid temperature at k beats T_k;
-    # the ECE of each candidate is the oracle's own ECE of the explicit product
+    # with T_1..T_{k-1} frozen, no grid temperature at k beats T_k; each candidate's
+    # ECE is the oracle's ECE of the explicitly formed product.  Run once frozen at
+    # the fit's own choices and once at other temperatures (T_fixed).
     z, acc = synth.calibration_set(800, 4, seed=4)
     grid = 0.5 + 0.01 * np.arange(451)
-    T, e = oracle_mod.sts_fit(z, acc)
-    P = np.ones(800)
-    for k in range(4):
-        eces = [oracle_mod.ece(P * special.expit(z[:, k].astype(np.float64) / t), acc, k + 1)
-                for t in grid]
-        i = int(np.argmin(eces))
-        assert T[k] == grid[i] and e[k] == pytest.approx(eces[i], abs=1e-15)
-        P = P * special.expit(z[:, k].astype(np.float64) / T[k])
+    T_own, _ = oracle_mod.sts_fit(z, acc)
+    for fixed in (None, T_own[::-1].copy() + 0.3):
+        T, e, G = oracle_mod.sts_fit(z, acc, T_fixed=fixed, return_grid=True)
+        frozen = T if fixed is None else fixed
+        P = np.ones(800)
+        for k in range(4):
+            eces = [oracle_mod.ece(P * special.expit(z[:, k].astype(np.float64) / t), acc, k + 1)
+                    for t in grid]
+            i = int(np.argmin(eces))
+            assert T[k] == grid[i] and e[k] == pytest.approx(eces[i], abs=1e-15)
+            np.testing.assert_allclose(G[k], eces, rtol=0, atol=1e-15)
+            P = P * special.expit(z[:, k].astype(np.float64) / frozen[k])
+        if fixed is not None:
+            assert not np.array_equal(T[1:], T_own[1:])     # the frozen prefix matters
 
 
 def test_sts_fit_recovers_the_true_temperature(oracle_mod):
