@@ -198,7 +198,10 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     }
 
     if (!dev->draft_attr_set) {
-        if (cudaFuncSetAttribute(D::markov_draft_kernel,
+        if (cudaFuncSetAttribute(D::markov_draft_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 D::kDynSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(D::markov_draft_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  D::kDynSmem) != cudaSuccess)
             return DSPARK_CUDA_ERROR;
@@ -246,7 +249,9 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel, tm_w2, tm_u, prm));
+    if (M == 64)
+        return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64>, tm_w2, tm_u, prm));
+    return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128>, tm_w2, tm_u, prm));
 }
 
 int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x, const void *W1,

@@ -347,6 +347,99 @@ __device__ __forceinline__ void box_update(RowBest &best, const uint32_t (&a0)[3
     }
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+// M = 64 (rows 16q..16q+15 of the tile in TMEM lanes 32q..32q+15): one 64-column box
+// read with 16x256b loads, so all 32 lanes work.  Thread t holds rows ra = t/4 and
+// rb = t/4 + 8 of the quadrant and, of the box, columns 8i + 2(t%4) + e (i = 0..7,
+// e = 0, 1): a[4i + e] is row ra, a[4i + 2 + e] row rb.  Each thread keeps a running
+// best per row over its own columns; the four threads of a row are combined by the
+// caller.  `two` is false when the box's second 32 columns lie outside the tile.
+__device__ __forceinline__ void box_update_m64(RowBest (&best)[2], const uint32_t (&a)[32],
+                                               bool two, uint32_t sU, int ua, int ub, int v0,
+                                               const Params &p, int k, int bg_a, int bg_b)
+{
+    const int w = threadIdx.x & 3;
+    float l[32], s[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t wa = lds32(sU + ua * 128 + ((i ^ (ua & 7)) << 4) + w * 4);
+        const uint32_t wb = lds32(sU + ub * 128 + ((i ^ (ub & 7)) << 4) + w * 4);
+        l[4 * i + 0] = __uint_as_float(a[4 * i + 0]) + bf16lo_to_f32(wa);
+        l[4 * i + 1] = __uint_as_float(a[4 * i + 1]) + bf16hi_to_f32(wa);
+        l[4 * i + 2] = __uint_as_float(a[4 * i + 2]) + bf16lo_to_f32(wb);
+        l[4 * i + 3] = __uint_as_float(a[4 * i + 3]) + bf16hi_to_f32(wb);
+    }
+    const int vw = v0 + 2 * w;                    // column of a[0]
+    if (!two || v0 + 2 * kUnit > p.V) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                if ((!two && i >= 4) || vw + 8 * i + e >= p.V) {
+                    l[4 * i + e] = -INFINITY;
+                    l[4 * i + 2 + e] = -INFINITY;
+                }
+    }
+    if (p.mode == 0) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = l[j];
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float lmax = fmaxf(l[4 * i + 2 * h], l[4 * i + 2 * h + 1]);
+                // exact pruning: noise cannot lift this pair above the row's running best
+                const bool skip = !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best[h].s);
+                if (__all_sync(0xFFFFFFFFu, skip)) {
+                    s[4 * i + 2 * h] = s[4 * i + 2 * h + 1] = -INFINITY;
+                } else {
+                    const uint4 g = philox(make_uint4(static_cast<uint32_t>((vw + 8 * i) >> 2),
+                                                      static_cast<uint32_t>(k - 1),
+                                                      static_cast<uint32_t>(h ? bg_b : bg_a), 0u),
+                                           p.seed_lo, p.seed_hi);
+                    const uint32_t g0 = (w & 1) ? g.z : g.x, g1 = (w & 1) ? g.w : g.y;
+                    s[4 * i + 2 * h] = fmaf(l[4 * i + 2 * h], p.inv_tau, gumbel_from_word(g0));
+                    s[4 * i + 2 * h + 1] = fmaf(l[4 * i + 2 * h + 1], p.inv_tau, gumbel_from_word(g1));
+                    if (skip) s[4 * i + 2 * h] = s[4 * i + 2 * h + 1] = -INFINITY;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float m4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            m4[i] = fmaxf(fmax3(s[8 * i + 2 * h], s[8 * i + 2 * h + 1], s[8 * i + 4 + 2 * h]),
+                          s[8 * i + 4 + 2 * h + 1]);
+        const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+        if (mx > best[h].s) {
+            int idx = 31;
+#pragma unroll
+            for (int i = 7; i >= 0; --i)
+#pragma unroll
+                for (int e = 1; e >= 0; --e)
+                    if (s[4 * i + 2 * h + e] == mx) idx = 4 * i + 2 * h + e;
+            float li = l[2 * h];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j == idx) li = l[j];
+            best[h].v = static_cast<uint32_t>(vw + 8 * (idx >> 2) + (idx & 1));
+            best[h].l = li;
+            best[h].s = mx;
+        }
+    }
+}
+
+// kM is the MMA's M (64 when B <= 64, else 128); p.M equals it.
+template <int kM>
 __global__ void __launch_bounds__(kThreads, 1)
     markov_draft_kernel(const __grid_constant__ CUtensorMap tm_w2,
                         const __grid_constant__ CUtensorMap tm_u, const Params p)
@@ -356,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int M = p.M;
+    constexpr int M = kM;
     const int a_chunk = M * 128;                  // one 64-column K chunk of A
     const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     const uint32_t sA = base;
@@ -573,6 +666,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         int next_tok[kMaxMTiles];
         unsigned long long my_key[kMaxMTiles];
         float my_logit[kMaxMTiles];
+        // M = 64 (one M tile): this thread's rows ra = lane/4 and rb = lane/4 + 8 of the quadrant
+        const int r64 = q * 16 + (lane >> 2);
+        const int ua64 = min(r64, p.ub - 1), ub64 = min(r64 + 8, p.ub - 1);
+        unsigned long long key64[2] = {0ull, 0ull};
+        float logit64[2] = {0.0f, 0.0f};
         for (int mt = 0; mt < num_mt; ++mt) {
             const int b = mt * M + row;
             next_tok[mt] = (lane_row && b < p.B) ? checked_token(p.anchor[b], p.V) : -1;
@@ -618,6 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool active = (m0 + q * rq) < p.B;
                 const int b_glob = my_b + p.b_offset;
                 RowBest best;
+                RowBest best64[2];
                 for (int t = 0; t < ntiles && ok; ++t) {
                     int first, count;
                     tile_span(t, n_units, ntiles, first, count);
@@ -645,7 +744,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 15, globaltimer_ns() - tw2);
-                        if (active) {
+                        if (active && M == 64) {
+                            uint32_t a[32];
+                            tmem_ld_16x256b_x8(t_acc + 2 * i * kUnit, a);
+                            tmem_wait_ld();
+                            box_update_m64(best64, a, 2 * i + 1 < count, sU + slot * p.u_slot_bytes,
+                                           ua64, ub64, (u_begin + first + 2 * i) * kUnit, p, k,
+                                           r64 + p.b_offset, r64 + 8 + p.b_offset);
+                        } else if (active) {
                             const bool two = 2 * i + 1 < count;
                             uint32_t a0[32], a1[32];
                             tmem_ld_32x32b_x32(t_acc + 2 * i * kUnit, a0);
@@ -678,7 +784,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     gather(mt + 1);
                 }
-                if (lane_row && my_b < p.B) {
+                if (M == 64) {
+                    // the four threads of a row hold disjoint columns: combine, one atomic per row
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const unsigned long long key = argmax_key(best64[h].s, best64[h].v);
+                        key64[h] = key;
+                        logit64[h] = best64[h].l;
+                        unsigned long long kr = key;
+                        kr = max(kr, __shfl_xor_sync(0xFFFFFFFFu, kr, 1));
+                        kr = max(kr, __shfl_xor_sync(0xFFFFFFFFu, kr, 2));
+                        const int b = r64 + 8 * h;
+                        if ((lane & 3) == 0 && b < p.B)
+                            atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + b], kr);
+                    }
+                } else if (lane_row && my_b < p.B) {
                     const unsigned long long key = argmax_key(best.s, best.v);
                     atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + my_b], key);
                     my_key[mt] = key;
@@ -720,9 +840,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const unsigned long long key = __ldcg(&p.slots[o]);
                 const int tok = static_cast<int>(argmax_key_index(key));
                 next_tok[mt] = checked_token(tok, p.V);
-                if (key == my_key[mt]) {
+                if (M != 64 && key == my_key[mt]) {
                     p.x_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = tok;
                     p.logit_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = my_logit[mt];
+                }
+            }
+            if (M == 64) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int b = r64 + 8 * h;
+                    if (b >= p.B) continue;
+                    const size_t o = static_cast<size_t>(k - 1) * p.B + b;
+                    const unsigned long long key = __ldcg(&p.slots[o]);
+                    if (key == key64[h]) {
+                        p.x_out[static_cast<size_t>(b) * p.gamma + (k - 1)] =
+                            static_cast<int>(argmax_key_index(key));
+                        p.logit_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = logit64[h];
+                    }
                 }
             }
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 6);

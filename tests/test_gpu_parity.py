@@ -174,6 +174,10 @@ STRESS = [
                    logits="zipf", mode=1, tau=0.7),
     synth.Workload("stress B=9 V=40000 gumbel", B=9, gamma=5, V=40000, d=64, w_std=0.2,
                    logits="normal", mode=1, tau=1.3, seed=5),
+    # M = 64 tiles with 1- and 2-unit CTAs, a ragged vocabulary tail and a full 64-row tile
+    synth.Workload("stress B=33 V=9000 gumbel", B=33, gamma=4, V=9000, d=64, w_std=0.2,
+                   logits="normal", mode=1, tau=0.9, seed=3),
+    synth.Workload("stress B=64 V=4104", B=64, gamma=5, V=4104, d=64, w_std=0.2, seed=2),
 ]
 
 
