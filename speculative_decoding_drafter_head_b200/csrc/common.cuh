@@ -15,20 +15,20 @@ __device__ __forceinline__ void record_error(unsigned int code)
 }
 
 // Optional timeline trace of the draft kernel (build with -DDSPARK_TRACE): per CTA and
-// per position k, 16 slots of %globaltimer stamps or accumulated wait times in ns.
+// per position k, 32 slots of %globaltimer stamps or accumulated wait times in ns.
 #ifdef DSPARK_TRACE
-__device__ unsigned long long g_trace[256 * 64 * 16];
+__device__ unsigned long long g_trace[256 * 64 * 32];
 #define DSPARK_TRACE_AT(k, slot)                                                              \
     do {                                                                                      \
         if ((k) <= 64 && blockIdx.x < 256) {                                                  \
             uint64_t t_;                                                                      \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                            \
-            g_trace[(blockIdx.x * 64 + ((k) - 1)) * 16 + (slot)] = t_;                        \
+            g_trace[(blockIdx.x * 64 + ((k) - 1)) * 32 + (slot)] = t_;                        \
         }                                                                                     \
     } while (0)
 #define DSPARK_TRACE_ADD(k, slot, v)                                                          \
     do {                                                                                      \
-        if ((k) <= 64 && blockIdx.x < 256) g_trace[(blockIdx.x * 64 + ((k) - 1)) * 16 + (slot)] += (v); \
+        if ((k) <= 64 && blockIdx.x < 256) g_trace[(blockIdx.x * 64 + ((k) - 1)) * 32 + (slot)] += (v); \
     } while (0)
 #else
 #define DSPARK_TRACE_AT(k, slot) \

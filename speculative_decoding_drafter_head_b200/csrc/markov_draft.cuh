@@ -590,6 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (mt == 0) DSPARK_TRACE_AT(k, 16);
                     tc_fence_after();
                     for (int t = 0; t < ntiles && ok; ++t) {
                         int first, count;
@@ -615,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 break;
                             }
                             DSPARK_TRACE_ADD(k, 13, globaltimer_ns() - tw1);
+                            if (mt == 0 && t == 0 && ks == 0) DSPARK_TRACE_AT(k, 17);
                             tc_fence_after();
                             // descriptors differ only in the start-address field (bits 0..13,
                             // 16-byte units): advance them with plain adds
@@ -720,6 +722,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < ntiles && ok; ++t) {
                     int first, count;
                     tile_span(t, n_units, ntiles, first, count);
+#ifdef DSPARK_TRACE
+                    const uint64_t tfw0 = globaltimer_ns();
+#endif
                     // warp-uniform outcome: tcgen05.ld below needs every lane of the warp
                     if (!__all_sync(0xFFFFFFFFu,
                                     wait_phase(bar_tfull + 8 * acc.slot, acc.phase, ctl, p))) {
@@ -728,6 +733,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     if (threadIdx.x == 0 && mt == 0 && t == 0) DSPARK_TRACE_AT(k, 2);
+                    if (threadIdx.x == 0 && mt == num_mt - 1 && t == ntiles - 1) DSPARK_TRACE_AT(k, 21);
+                    if (threadIdx.x == 0 && t > 0) DSPARK_TRACE_ADD(k, 20, globaltimer_ns() - tfw0);
+#ifdef DSPARK_TRACE
+                    const uint64_t tbusy0 = globaltimer_ns();
+#endif
                     // box i of the tile holds chunks 2i and 2i + 1; this warp takes boxes i = half,
                     // half + 2, ... and reduces both chunks of a box together
                     const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
@@ -764,6 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0) mbar_arrive(bar_u_empty + 8 * slot);
                     }
                     u_pos += nbox;
+                    if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 19, globaltimer_ns() - tbusy0);
                     if (!ok) break;
                     tc_fence_before();
                     __syncwarp();
