@@ -300,6 +300,9 @@ def main():
     ap.add_argument("--eager", action="store_true", help="launch kernels one by one (no CUDA graph)")
     ap.add_argument("--stage", default="path", choices=["path", "sts-fit"],
                     help="path: the per-step hot path; sts-fit: the temperature fit")
+    ap.add_argument("--schedule", default="sync", choices=["sync", "lagged"],
+                    help="sync: schedule on this step's scores; lagged: on the scores of two "
+                         "steps earlier, on a side stream that overlaps the draft kernel")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     if args.stage == "sts-fit":
@@ -366,8 +369,17 @@ def main():
     target = torch.from_numpy(target_h).cuda()
 
     ev_draft = []
+    lagged = args.schedule == "lagged"
+    lsched = None
+    last_L = [None]
+    if lagged:
+        from speculative_decoding_drafter_head_b200 import pipeline
+        lsched = pipeline.LaggedScheduler(B * world, gamma, Tstep, lag=2)
+    step_no = [0]
 
     def step(record=None):
+        t = step_no[0]
+        step_no[0] += 1
         e0 = e1 = None
         if record is not None:
             e0 = torch.cuda.Event(enable_timing=True)
@@ -378,37 +390,62 @@ def main():
         if record is not None:
             e1.record(stream)
             record.append((e0, e1))
-        ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P)
-        if world > 1:
-            sharding.gather_scores(P, out=Pg)
-            ds.schedule_prefix(Pg, Tstep, Lg, Nst, obj, ws)
-            Lloc = sharding.local_lengths(Lg, rank, B)
+        if lagged:
+            lsched.begin_step(t)                   # overlaps the confidence kernel
+            if world > 1:
+                ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P)
+                sharding.gather_scores(P, out=lsched.scores(t))
+            else:
+                ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, lsched.scores(t))
+            Lt = lsched.lengths(t, workspace=ws)
+            Lloc = sharding.local_lengths(Lt, rank, B) if world > 1 else Lt
         else:
-            ds.schedule_prefix(P, Tstep, Lg, Nst, obj, ws)
-            Lloc = Lg
+            ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P)
+            if world > 1:
+                sharding.gather_scores(P, out=Pg)
+                ds.schedule_prefix(Pg, Tstep, Lg, Nst, obj, ws)
+                Lloc = sharding.local_lengths(Lg, rank, B)
+            else:
+                ds.schedule_prefix(P, Tstep, Lg, Nst, obj, ws)
+                Lloc = Lg
         ds.verify_prefix(x, Lloc, target, acc, bonus)
+        last_L[0] = Lloc
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert ds.get_error() == 0, "device error during warm-up"
 
-    # one step as a CUDA graph (launch gaps removed); eager launches if capture is refused
-    graph = None
+    # one step as a CUDA graph (launch gaps removed); eager launches if capture is refused.
+    # The lagged schedule rotates through 3 ring slots, so it needs one graph per slot.
+    graphs, graph_L = [], []
     if not args.eager:
         try:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                step()
-            g.replay()
+            for _ in range(3 if lagged else 1):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    step()
+                graphs.append(g)
+                graph_L.append(last_L[0])
+            for g in graphs:
+                g.replay()
             torch.cuda.synchronize()
             assert ds.get_error() == 0
-            graph = g
         except Exception as exc:                        # noqa: BLE001
             print(f"# CUDA graph capture unavailable, timing eager launches: {exc}",
                   file=sys.stderr)
             torch.cuda.synchronize()
-    run_step = graph.replay if graph is not None else step
+            graphs = []
+    graph = graphs[0] if graphs else None
+    replay_no = [0]
+
+    def replay():
+        j = replay_no[0] % len(graphs)
+        graphs[j].replay()
+        last_L[0] = graph_L[j]                     # the lengths this step verified with
+        replay_no[0] += 1
+
+    run_step = replay if graphs else step
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -458,7 +495,7 @@ def main():
         target.copy_(target_pin, non_blocking=True)
         run_step()
         out_x.copy_(x, non_blocking=True)
-        out_L.copy_(sharding.local_lengths(Lg, rank, B) if world > 1 else Lg, non_blocking=True)
+        out_L.copy_(last_L[0], non_blocking=True)
         out_acc.copy_(acc, non_blocking=True)
         out_bonus.copy_(bonus, non_blocking=True)
 
@@ -525,11 +562,13 @@ def main():
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": 4 * args.steps,
             "cuda_graph": graph is not None,
+            "schedule": "lagged by 2 steps, side stream" if lagged else "this step's scores",
             "clocks": clk,
             "draft_kernel_ms": {"mean": draft_mean, "min": min(draft_ms), "max": max(draft_ms)},
         }
         print(json.dumps(line), flush=True)
-    graph = None                                    # release the graph before the group
+    graph = None                                    # release the graphs before the group
+    graphs = []
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
