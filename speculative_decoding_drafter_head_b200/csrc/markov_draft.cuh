@@ -277,24 +277,25 @@ __device__ __forceinline__ void scores32(float (&s)[32], float (&l)[32], int v0,
         for (int i = 0; i < 32; ++i) s[i] = l[i];
         return;
     }
+    // exact pruning, one warp vote per chunk: skip the noise only when no lane's chunk can
+    // beat its running best even with the largest noise value; otherwise the eight Philox
+    // blocks run without branches so that their round chains interleave
+    const bool skip = !(fmaf(max32(l), p.inv_tau, kGumbelMax) >= best_s);
+    if (__all_sync(0xFFFFFFFFu, skip)) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] = -INFINITY;
+        return;
+    }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        const float lmax = fmaxf(fmaxf(l[4 * q], l[4 * q + 1]), fmaxf(l[4 * q + 2], l[4 * q + 3]));
-        // exact pruning: noise cannot lift this group above the running best
-        const bool skip = !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best_s);
-        if (__all_sync(0xFFFFFFFFu, skip)) {
-            s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
-        } else {
-            const uint4 w = philox(make_uint4(static_cast<uint32_t>(v0 / 4 + q),
-                                              static_cast<uint32_t>(k - 1),
-                                              static_cast<uint32_t>(b_glob), 0u),
-                                   p.seed_lo, p.seed_hi);
-            s[4 * q + 0] = fmaf(l[4 * q + 0], p.inv_tau, gumbel_from_word(w.x));
-            s[4 * q + 1] = fmaf(l[4 * q + 1], p.inv_tau, gumbel_from_word(w.y));
-            s[4 * q + 2] = fmaf(l[4 * q + 2], p.inv_tau, gumbel_from_word(w.z));
-            s[4 * q + 3] = fmaf(l[4 * q + 3], p.inv_tau, gumbel_from_word(w.w));
-            if (skip) s[4 * q] = s[4 * q + 1] = s[4 * q + 2] = s[4 * q + 3] = -INFINITY;
-        }
+        const uint4 w = philox(make_uint4(static_cast<uint32_t>(v0 / 4 + q),
+                                          static_cast<uint32_t>(k - 1),
+                                          static_cast<uint32_t>(b_glob), 0u),
+                               p.seed_lo, p.seed_hi);
+        s[4 * q + 0] = fmaf(l[4 * q + 0], p.inv_tau, gumbel_from_word(w.x));
+        s[4 * q + 1] = fmaf(l[4 * q + 1], p.inv_tau, gumbel_from_word(w.y));
+        s[4 * q + 2] = fmaf(l[4 * q + 2], p.inv_tau, gumbel_from_word(w.z));
+        s[4 * q + 3] = fmaf(l[4 * q + 3], p.inv_tau, gumbel_from_word(w.w));
     }
 }
 
@@ -390,25 +391,40 @@ __device__ __forceinline__ void box_update_m64(RowBest (&best)[2], const uint32_
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[j] = l[j];
     } else {
+        // one vote per box: skip the noise only when no thread's columns can beat its row's
+        // running best even with the largest noise value
+        float lm0 = -INFINITY, lm1 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
+            lm0 = fmax3(lm0, l[4 * i + 0], l[4 * i + 1]);
+            lm1 = fmax3(lm1, l[4 * i + 2], l[4 * i + 3]);
+        }
+        const bool skip = !(fmaf(lm0, p.inv_tau, kGumbelMax) >= best[0].s) &&
+                          !(fmaf(lm1, p.inv_tau, kGumbelMax) >= best[1].s);
+        if (__all_sync(0xFFFFFFFFu, skip)) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float lmax = fmaxf(l[4 * i + 2 * h], l[4 * i + 2 * h + 1]);
-                // exact pruning: noise cannot lift this pair above the row's running best
-                const bool skip = !(fmaf(lmax, p.inv_tau, kGumbelMax) >= best[h].s);
-                if (__all_sync(0xFFFFFFFFu, skip)) {
-                    s[4 * i + 2 * h] = s[4 * i + 2 * h + 1] = -INFINITY;
-                } else {
-                    const uint4 g = philox(make_uint4(static_cast<uint32_t>((vw + 8 * i) >> 2),
-                                                      static_cast<uint32_t>(k - 1),
-                                                      static_cast<uint32_t>(h ? bg_b : bg_a), 0u),
-                                           p.seed_lo, p.seed_hi);
-                    const uint32_t g0 = (w & 1) ? g.z : g.x, g1 = (w & 1) ? g.w : g.y;
-                    s[4 * i + 2 * h] = fmaf(l[4 * i + 2 * h], p.inv_tau, gumbel_from_word(g0));
-                    s[4 * i + 2 * h + 1] = fmaf(l[4 * i + 2 * h + 1], p.inv_tau, gumbel_from_word(g1));
-                    if (skip) s[4 * i + 2 * h] = s[4 * i + 2 * h + 1] = -INFINITY;
-                }
+            for (int j = 0; j < 32; ++j) s[j] = -INFINITY;
+        } else {
+            // columns 8i + 2w + {0,1} are words 2(w&1) + {0,1} of Philox block 2i + (w>>1);
+            // threads w and w^1 need the same block for both rows, so each computes it for
+            // one row (w&1 ? rb : ra) and passes the other thread its two words
+            const int own_b = (w & 1) ? bg_b : bg_a;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 g = philox(make_uint4(static_cast<uint32_t>((v0 >> 2) + 2 * i + (w >> 1)),
+                                                  static_cast<uint32_t>(k - 1),
+                                                  static_cast<uint32_t>(own_b), 0u),
+                                       p.seed_lo, p.seed_hi);
+                const uint32_t send0 = (w & 1) ? g.x : g.z, send1 = (w & 1) ? g.y : g.w;
+                const uint32_t recv0 = __shfl_xor_sync(0xFFFFFFFFu, send0, 1);
+                const uint32_t recv1 = __shfl_xor_sync(0xFFFFFFFFu, send1, 1);
+                // row ra: own words when w is even, else the neighbour's; row rb the reverse
+                const uint32_t a0 = (w & 1) ? recv0 : g.x, a1 = (w & 1) ? recv1 : g.y;
+                const uint32_t b0 = (w & 1) ? g.z : recv0, b1 = (w & 1) ? g.w : recv1;
+                s[4 * i + 0] = fmaf(l[4 * i + 0], p.inv_tau, gumbel_from_word(a0));
+                s[4 * i + 1] = fmaf(l[4 * i + 1], p.inv_tau, gumbel_from_word(a1));
+                s[4 * i + 2] = fmaf(l[4 * i + 2], p.inv_tau, gumbel_from_word(b0));
+                s[4 * i + 3] = fmaf(l[4 * i + 3], p.inv_tau, gumbel_from_word(b1));
             }
         }
     }
