@@ -119,15 +119,16 @@ int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x
  * steps-per-second curve) and [G] section 6 ("global throughput maximization").
  *
  * Scores P[b, k-1] (non-increasing in k, within [0, 1]) are ordered by
- * (P desc, b asc, k asc); q = floor(P 2^48); S_N = sum of the first N q's;
- *   F(N) = double(B 2^48 + S_N) / Tstep_us[B + N],   N = 0 .. B gamma
- * (int64 sum, round-to-nearest conversion and division).  N* = smallest N with
+ * (P desc, b asc, k asc); q = floor(P 2^46); S_N = sum of the first N q's;
+ *   F(N) = double(B 2^46 + S_N) / Tstep_us[B + N],   N = 0 .. B gamma
+ * (int64 sum, which stays below (B + B gamma) 2^46 < 2^63 at every supported size;
+ * round-to-nearest conversion and division).  N* = smallest N with
  * the largest F; L_out[b] = number of request b's entries among the first N*.
  *
  *   P [B, gamma] fp32;  Tstep_us [B (gamma + 1) + 1] fp64, Tstep_us[n] > 0 is the
  *   time of one target step that verifies n tokens (each request feeds its
  *   anchor/bonus position plus L_b drafts, so n = B + sum L).
- *   L_out [B] int32;  N_out [1] int32 (N*);  objective_out [1] fp64 = F(N*) 2^-48,
+ *   L_out [B] int32;  N_out [1] int32 (N*);  objective_out [1] fp64 = F(N*) 2^-46,
  *   expected accepted tokens (bonus included) per unit of Tstep's time.
  * Supported sizes: 1 <= B <= 32768, 1 <= gamma <= 64, B gamma <= 65536.
  * A score outside [0, 1] or an increase along a request records

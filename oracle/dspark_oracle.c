@@ -35,7 +35,7 @@
  *     probabilities", [G] section 5: "cumulative product");
  *   - scheduler objective: expected tokens per second
  *     F = (B + sum_b sum_{k <= L_b} P_{b,k}) / Tstep(B + sum_b L_b), scores
- *     fixed-point q = floor(P 2^48), order (P desc, b asc, k asc), first
+ *     fixed-point q = floor(P 2^46), order (P desc, b asc, k asc), first
  *     maximum over N ([W]; [G] section 6);
  *   - verification: accepted = index of the first mismatch among the first L_b
  *     drafts (or L_b), bonus = target token at that position ([S]).
@@ -256,13 +256,15 @@ int oracle_confidence(const uint16_t *h, const int32_t *anchor, const int32_t *x
  * [G] section 6, "global throughput maximization").
  *
  * Scores P[b, k-1] (fp32) are ordered by (P desc, b asc, k asc).  With
- * q = floor(P 2^48) (exact integers) and S_N the sum of the first N of them,
- *   F(N) = double(B 2^48 + S_N) / Tstep[B + N],     N = 0 .. B gamma,
+ * q = floor(P 2^46) (exact integers) and S_N the sum of the first N of them,
+ *   F(N) = double(B 2^46 + S_N) / Tstep[B + N],     N = 0 .. B gamma,
  * N* is the smallest N with the largest F, and L_b counts the entries of
  * request b among the first N*.  Tstep[n] is the wall time of one target step
  * that verifies n tokens (each request feeds its anchor plus L_b drafts).
- * The reported objective is F 2^-48 (an exact rescaling): expected accepted
- * tokens per unit of Tstep's time.
+ * The reported objective is F 2^-46 (an exact rescaling): expected accepted
+ * tokens per unit of Tstep's time.  The scale 2^46 keeps the largest numerator,
+ * (B + B gamma) 2^46 <= 98304 2^46 < 2^63, inside int64 for every supported size
+ * (B <= 32768, B gamma <= 65536).
  * ------------------------------------------------------------------------ */
 typedef struct {
     float p;
@@ -306,17 +308,17 @@ int oracle_schedule(const float *P, int B, int gamma, const double *Tstep, int32
         }
     qsort(s, (size_t)n, sizeof(oracle_score_t), score_order);
 
-    const int64_t base = (int64_t)B << 48;
+    const int64_t base = (int64_t)B << 46;
     int64_t S = 0;
     double bestF = (double)base / Tstep[B];
     int bestN = 0;
     if (F_all)
-        F_all[0] = ldexp(bestF, -48);
+        F_all[0] = ldexp(bestF, -46);
     for (int N = 1; N <= n; ++N) {
-        S += (int64_t)floor(ldexp((double)s[N - 1].p, 48));
+        S += (int64_t)floor(ldexp((double)s[N - 1].p, 46));
         const double F = (double)(base + S) / Tstep[B + N];
         if (F_all)
-            F_all[N] = ldexp(F, -48);
+            F_all[N] = ldexp(F, -46);
         if (F > bestF) {
             bestF = F;
             bestN = N;
@@ -329,7 +331,7 @@ int oracle_schedule(const float *P, int B, int gamma, const double *Tstep, int32
     if (N_out)
         *N_out = bestN;
     if (F_out)
-        *F_out = ldexp(bestF, -48);
+        *F_out = ldexp(bestF, -46);
     free(s);
     return ORACLE_OK;
 }

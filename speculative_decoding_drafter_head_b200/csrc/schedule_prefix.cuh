@@ -11,9 +11,10 @@
 // (P desc, b asc, k asc) -- each request's row is already in that order, so the rank
 // of (b, k) is the sum over rows b' of a binary search in row b'.  Phase 2 (the last
 // CTA to finish, found with a completion counter, no spinning): scatter the
-// fixed-point scores q = floor(P 2^48) into rank order, prefix-sum them in int64,
-// evaluate F(N) = double(B 2^48 + S_N) / Tstep[B + N] for every N, take the first
-// maximum, and count each request's entries below it.
+// fixed-point scores q = floor(P 2^46) into rank order, prefix-sum them in int64,
+// evaluate F(N) = double(B 2^46 + S_N) / Tstep[B + N] for every N, take the first
+// maximum, and count each request's entries below it.  With B <= 32768 and
+// B gamma <= 65536 the numerator stays below (B + B gamma) 2^46 < 2^63.
 #pragma once
 #include "common.cuh"
 
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params 
     for (int i = threadIdx.x; i < p.n; i += kThreads) {
         const int pos = __ldcg(p.rank + i);
         const float pi = __ldg(p.P + i);
-        p.q_sorted[pos] = __float2ll_rz(pi * 0x1p48f);
+        p.q_sorted[pos] = __float2ll_rz(pi * 0x1p46f);
     }
     __syncthreads();
 
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params 
     long long total;
     long long S = block_exclusive_scan(part, s_warp, total);
 
-    const long long base = static_cast<long long>(p.B) << 48;
+    const long long base = static_cast<long long>(p.B) << 46;
     double best = -1.0;
     int bestN = 0;
     if (threadIdx.x == 0) {
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params 
             }
         }
         *p.N_out = s_bestN[0];
-        *p.objective_out = s_bestF[0] * 0x1p-48;
+        *p.objective_out = s_bestF[0] * 0x1p-46;
         *p.done = 0u;
     }
     __syncthreads();

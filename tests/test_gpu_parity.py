@@ -73,7 +73,7 @@ def _tstep(kind, B, gamma, rng):
 
 
 SCHED_CASES = [(1, 1), (1, 16), (3, 4), (4, 8), (37, 13), (64, 16), (256, 16), (512, 16),
-               (1024, 24), (2048, 32)]
+               (1024, 24), (2048, 32), (1024, 64), (32768, 2)]     # the last two: largest B*gamma, gamma, B
 
 
 @pytest.mark.parametrize("B,gamma", SCHED_CASES)
@@ -110,10 +110,14 @@ def test_schedule_records_increasing_scores(ds):
 
 
 # ---------------------------------------------------------------------------- confidence
-@pytest.mark.parametrize("name", ["tiny", "qwen3-8b", "large-vocab-part"])
+_CONF_EXTRA = {"large-vocab-part": synth.LARGE_VOCAB.with_(B=96),
+               "gamma64": synth.Workload("conf B=5 gamma=64 d=256", B=5, gamma=64, V=1000, d=256)}
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3-8b", "large-vocab-part", "gamma64"])
 def test_confidence_within_tolerance(ds, oracle_mod, name):
     import torch
-    wl = synth.WORKLOADS[name] if name != "large-vocab-part" else synth.LARGE_VOCAB.with_(B=96)
+    wl = _CONF_EXTRA.get(name) or synth.WORKLOADS[name]
     W1 = synth.w1(wl)
     h = synth.h_all(wl)
     anchor = synth.anchors(wl)
@@ -178,6 +182,10 @@ STRESS = [
     synth.Workload("stress B=33 V=9000 gumbel", B=33, gamma=4, V=9000, d=64, w_std=0.2,
                    logits="normal", mode=1, tau=0.9, seed=3),
     synth.Workload("stress B=64 V=4104", B=64, gamma=5, V=4104, d=64, w_std=0.2, seed=2),
+    # the largest gamma the kernel takes, one row and a 130-row tile pair
+    synth.Workload("stress B=3 gamma=64 V=2048", B=3, gamma=64, V=2048, d=64, w_std=0.3, seed=4),
+    synth.Workload("stress B=130 gamma=64 V=1032", B=130, gamma=64, V=1032, d=64, w_std=0.3,
+                   seed=6),
 ]
 
 

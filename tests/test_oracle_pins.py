@@ -244,11 +244,11 @@ def test_confidence_rejects_bad_temperature(oracle_mod):
 def _objective(P, L, Tstep):
     """Expected tokens per second of a verify-length choice, exact numerator."""
     B = P.shape[0]
-    num = B << 48
+    num = B << 46
     for b in range(B):
         for k in range(L[b]):
-            num += math.floor(float(P[b, k]) * 2.0**48)
-    return math.ldexp(float(num) / float(Tstep[B + sum(L)]), -48)
+            num += math.floor(float(P[b, k]) * 2.0**46)
+    return math.ldexp(float(num) / float(Tstep[B + sum(L)]), -46)
 
 
 def _tables(B, gamma, rng):
@@ -278,6 +278,20 @@ def test_schedule_matches_brute_force_enumeration(oracle_mod, B, gamma):
             assert F == best
             assert _objective(P, L, Tstep) == best
             assert N == int(L.sum()) == best_n
+
+
+@pytest.mark.parametrize("B,gamma", [(32768, 2), (1024, 64)])
+def test_schedule_largest_sizes_closed_form(oracle_mod, B, gamma):
+    # every score 1 and a flat curve: verify everything, F = (B + B gamma) / T exactly.
+    # The fixed-point numerator (B + B gamma) 2^46 must not overflow at these sizes.
+    T = 15000.0
+    L, N, F, _ = oracle_mod.schedule(np.ones((B, gamma), np.float32), np.full(B * (gamma + 1) + 1, T))
+    assert (L == gamma).all() and N == B * gamma
+    assert F == (B + B * gamma) / T
+    # halve every score: F = (B + B gamma / 2) / T, still everything verified
+    L, N, F, _ = oracle_mod.schedule(np.full((B, gamma), 0.5, np.float32),
+                                     np.full(B * (gamma + 1) + 1, T))
+    assert N == B * gamma and F == (B + B * gamma / 2) / T
 
 
 def test_schedule_flat_curve_verifies_everything(oracle_mod):
