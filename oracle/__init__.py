@@ -46,6 +46,9 @@ def _load():
         lib.oracle_draft.argtypes = [p, p, p, p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                      C.c_double, C.c_uint64, p, p, p, p, C.c_int]
         lib.oracle_draft.restype = C.c_int
+        lib.oracle_draft_rnn.argtypes = [p, p, p, p, p, C.c_int, C.c_int, C.c_int, C.c_int,
+                                         C.c_int, C.c_double, C.c_uint64, p, p, p, p, C.c_int]
+        lib.oracle_draft_rnn.restype = C.c_int
         lib.oracle_confidence.argtypes = [p, p, p, p, p, C.c_double, p, C.c_int, C.c_int,
                                           C.c_int, C.c_int, C.c_int, p, p, p, p, C.c_int]
         lib.oracle_confidence.restype = C.c_int
@@ -110,6 +113,29 @@ def draft(U, anchor, W1, W2, mode: int = 0, tau: float = 1.0, seed: int = 0, b_i
                               _ptr(logit), _ptr(gap), int(nthreads))
     if st != 0:
         raise ValueError(f"oracle_draft rejected its arguments (status {st})")
+    return x, logit, gap
+
+
+def draft_rnn(U, anchor, W1, W2, Whh, mode: int = 0, tau: float = 1.0, seed: int = 0,
+              b_index=None, nthreads: int = 0):
+    """RNN-head drafting (Elman reading); returns (x, logit, gap) as draft()."""
+    U = _c(U, np.uint16)
+    nb, gamma, V = U.shape
+    W1 = _c(W1, np.uint16)
+    W2 = _c(W2, np.uint16)
+    Whh = _c(Whh, np.uint16)
+    r = W1.shape[1]
+    assert W1.shape == (V, r) and W2.shape == (r, V) and Whh.shape == (r, r)
+    anchor = _c(anchor, np.int32)
+    bi = _c(np.arange(nb) if b_index is None else b_index, np.int32)
+    x = np.zeros((nb, gamma), dtype=np.int32)
+    logit = np.zeros((nb, gamma), dtype=np.float64)
+    gap = np.zeros((nb, gamma), dtype=np.float64)
+    st = _load().oracle_draft_rnn(_ptr(U), _ptr(anchor), _ptr(W1), _ptr(W2), _ptr(Whh), nb,
+                                  gamma, V, r, int(mode), float(tau), int(seed) & (2**64 - 1),
+                                  _ptr(bi), _ptr(x), _ptr(logit), _ptr(gap), int(nthreads))
+    if st != 0:
+        raise ValueError(f"oracle_draft_rnn rejected its arguments (status {st})")
     return x, logit, gap
 
 

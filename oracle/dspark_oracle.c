@@ -189,6 +189,107 @@ int oracle_draft(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
 }
 
 /* --------------------------------------------------------------------------
+ * RNN head ([G] section 4, "Two instantiations of the sequential block": a
+ * recurrent state that accumulates the whole prefix of the block).  The pages
+ * give no equations; this is the plain Elman reading over the Markov head's
+ * factors (PARITY UNPINNED against the pages):
+ *   s_0 = 0,   s_k = tanh(W1[x_{k-1}] + s_{k-1} Whh)       (r-vector, fp64)
+ *   a_k = bf16(fp32(s_k))                                   (the GEMM operand)
+ *   l_k(v) = U[b, k-1, v] + sum_j a_k[j] W2[j, v]
+ * and x_k is chosen as in oracle_draft (greedy or Gumbel-max).  With Whh = 0
+ * the bias is that of a Markov head whose table is bf16(fp32(tanh(W1))).
+ * ------------------------------------------------------------------------ */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu))
+        return (uint16_t)((u >> 16) | 0x40u);                  /* quiet NaN */
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+int oracle_draft_rnn(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
+                     const uint16_t *W2, const uint16_t *Whh, int nb, int gamma, int V, int r,
+                     int mode, double tau, uint64_t seed, const int32_t *b_index,
+                     int32_t *x_out, double *logit_out, double *gap_out, int nthreads)
+{
+    if (nb < 0 || gamma < 1 || V < 2 || r < 1 || (mode != 0 && mode != 1))
+        return ORACLE_INVALID;
+    if (mode == 1 && !(tau > 0.0))
+        return ORACLE_INVALID;
+    for (int i = 0; i < nb; ++i)
+        if (anchor[i] < 0 || anchor[i] >= V)
+            return ORACLE_INVALID;
+    if (nthreads < 1)
+        nthreads = oracle_num_threads();
+
+    int status = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int i = 0; i < nb; ++i) {
+        double *bias = (double *)malloc(sizeof(double) * (size_t)V);
+        double *st = (double *)calloc((size_t)r, sizeof(double));
+        double *nx = (double *)malloc(sizeof(double) * (size_t)r);
+        if (!bias || !st || !nx) {
+            free(bias);
+            free(st);
+            free(nx);
+#pragma omp atomic write
+            status = ORACLE_INVALID;
+            continue;
+        }
+        int prev = anchor[i];
+        for (int k = 1; k <= gamma; ++k) {
+            const uint16_t *row = W1 + (size_t)prev * (size_t)r;
+            for (int j = 0; j < r; ++j) {
+                double acc = bf16_to_f64(row[j]);
+                for (int q = 0; q < r; ++q)
+                    acc += st[q] * bf16_to_f64(Whh[(size_t)q * (size_t)r + (size_t)j]);
+                nx[j] = tanh(acc);
+            }
+            for (int j = 0; j < r; ++j)
+                st[j] = nx[j];
+            for (int v = 0; v < V; ++v)
+                bias[v] = 0.0;
+            for (int j = 0; j < r; ++j) {
+                const double a = bf16_to_f64(f32_to_bf16_rne((float)st[j]));
+                const uint16_t *w2j = W2 + (size_t)j * (size_t)V;
+                for (int v = 0; v < V; ++v)
+                    bias[v] += a * bf16_to_f64(w2j[v]);
+            }
+            const uint16_t *Uk = U + ((size_t)i * (size_t)gamma + (size_t)(k - 1)) * (size_t)V;
+            double best = -INFINITY, second = -INFINITY, best_l = 0.0;
+            int best_v = -1;
+            for (int v = 0; v < V; ++v) {
+                const double l = bf16_to_f64(Uk[v]) + bias[v];
+                double sc = l;
+                if (mode == 1)
+                    sc = l / tau + oracle_gumbel(seed, b_index ? b_index[i] : i, k, v);
+                if (sc > best) {
+                    second = best;
+                    best = sc;
+                    best_v = v;
+                    best_l = l;
+                } else if (sc > second) {
+                    second = sc;
+                }
+            }
+            const size_t o = (size_t)i * (size_t)gamma + (size_t)(k - 1);
+            x_out[o] = best_v;
+            if (logit_out)
+                logit_out[o] = best_l;
+            if (gap_out)
+                gap_out[o] = best - second;
+            prev = best_v;
+        }
+        free(bias);
+        free(st);
+        free(nx);
+    }
+    return status;
+}
+
+/* --------------------------------------------------------------------------
  * Confidence head, Sequential Temperature Scaling and prefix survival
  * ([G] section 5; [S] "Confidence-scheduled verification").
  *

@@ -481,3 +481,56 @@ def test_sts_fit_rejects_bad_arguments(oracle_mod):
         oracle_mod.sts_fit(z, acc, t_min=0.0)
     with pytest.raises(ValueError):
         oracle_mod.sts_fit(z, acc, n_bins=0)
+
+
+# ---------------------------------------------------------------------------
+# RNN head (gdymind.com "DSpark", section 4, second instantiation of the sequential
+# block: a recurrent state over the block's prefix).  No equations on the pages: the
+# Elman reading s_k = tanh(W1[x_{k-1}] + s_{k-1} Whh), bias = bf16(s_k) W2 is pinned
+# only by its special cases (parity unpinned against the pages).
+# ---------------------------------------------------------------------------
+def _rnn_inputs(nb, gamma, V, r, seed, whh_std):
+    U, anchor, W1, W2 = _tiny_draft_inputs(nb, gamma, V, r, 0.5, seed=seed)
+    rng = np.random.default_rng(seed + 1)
+    Whh = _bf16(rng.normal(0, whh_std, (r, r)))
+    return U, anchor, W1, W2, Whh
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_rnn_without_recurrence_is_a_markov_head_on_tanh_table(oracle_mod, mode):
+    # Whh = 0: s_k = tanh(W1[x_{k-1}]), so the RNN head drafts exactly like the Markov
+    # head whose table is bf16(fp32(tanh(W1)))
+    V, r, gamma, nb = 300, 16, 6, 4
+    U, anchor, W1, W2, _ = _rnn_inputs(nb, gamma, V, r, 5, 0.0)
+    Z = np.zeros((r, r), np.uint16)
+    W1t = synth.f32_to_bf16_bits(np.tanh(_f(W1)).astype(np.float32))
+    x_r, l_r, g_r = oracle_mod.draft_rnn(U, anchor, W1, W2, Z, mode=mode, tau=0.8, seed=3)
+    x_m, l_m, g_m = oracle_mod.draft(U, anchor, W1t, W2, mode=mode, tau=0.8, seed=3)
+    np.testing.assert_array_equal(x_r, x_m)
+    np.testing.assert_array_equal(l_r, l_m)
+    np.testing.assert_array_equal(g_r, g_m)
+
+
+def test_rnn_state_carries_the_prefix_beyond_the_last_token(oracle_mod):
+    # two requests with different anchors are forced to the same x_1 by a large base
+    # logit; at position 2 the Markov head (Whh = 0) then sees identical inputs, the RNN
+    # head does not: its state still holds the anchor
+    V, r, gamma = 64, 8, 2
+    U, _, W1, W2, Whh = _rnn_inputs(2, gamma, V, r, 9, 0.8)
+    Uf = np.zeros((2, gamma, V), np.float32)
+    Uf[:, 0, 7] = 50.0                                  # x_1 = 7 for both requests
+    U = synth.f32_to_bf16_bits(Uf)
+    anchor = np.array([3, 40], np.int32)
+    Z = np.zeros((r, r), np.uint16)
+    x0, l0, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Z)
+    x1, l1, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh)
+    assert (x0[:, 0] == 7).all() and (x1[:, 0] == 7).all()
+    assert x0[0, 1] == x0[1, 1] and l0[0, 1] == l0[1, 1]           # Markov: no memory
+    assert l1[0, 1] != l1[1, 1]                                    # RNN: the anchor persists
+
+
+def test_rnn_rejects_bad_anchor(oracle_mod):
+    U, anchor, W1, W2, Whh = _rnn_inputs(2, 3, 50, 4, 1, 0.1)
+    anchor[1] = 50
+    with pytest.raises(ValueError):
+        oracle_mod.draft_rnn(U, anchor, W1, W2, Whh)
