@@ -125,13 +125,17 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def cpu_oracle_step(wl, inp, bs, target_rows, oracle):
+def cpu_oracle_step(wl, inp, bs, target_rows, oracle, Whh=None):
     """The oracle's whole path on the listed requests (one bounded sample of a step)."""
     bs = list(bs)
     U = synth.u_requests(wl, bs) if inp.U is None else inp.U[bs]
     h = synth.h_requests(wl, bs) if inp.h is None else inp.h[bs]
-    x, _, _ = oracle.draft(U, inp.anchor[bs], inp.W1, inp.W2, mode=wl.mode, tau=wl.tau,
-                           seed=wl.seed, b_index=np.array(bs, np.int32))
+    if Whh is None:
+        x, _, _ = oracle.draft(U, inp.anchor[bs], inp.W1, inp.W2, mode=wl.mode, tau=wl.tau,
+                               seed=wl.seed, b_index=np.array(bs, np.int32))
+    else:
+        x, _, _ = oracle.draft_rnn(U, inp.anchor[bs], inp.W1, inp.W2, Whh, mode=wl.mode,
+                                   tau=wl.tau, seed=wl.seed, b_index=np.array(bs, np.int32))
     conf = oracle.confidence(h, inp.anchor[bs], x, inp.W1, inp.w, inp.b_conf, inp.T)
     sub = wl.with_(B=len(bs))
     L, _, _, _ = oracle.schedule(conf["P32"], synth.tstep_us(sub))
@@ -175,7 +179,7 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(wl, inp, target, budget_s):
+def cpu_baseline(wl, inp, target, budget_s, Whh=None):
     """Time the oracle's whole step on the host cores for about budget_s seconds.
 
     The sample grows from one request to the whole batch; when the whole batch takes
@@ -186,7 +190,7 @@ def cpu_baseline(wl, inp, target, budget_s):
     n = 1
     while True:
         t0 = time.perf_counter()
-        cpu_oracle_step(wl, inp, list(range(n)), target[:n], oracle)
+        cpu_oracle_step(wl, inp, list(range(n)), target[:n], oracle, Whh)
         dt = time.perf_counter() - t0
         if n >= wl.B or dt >= budget_s / 4:
             break
@@ -194,7 +198,7 @@ def cpu_baseline(wl, inp, target, budget_s):
     reps, total = 1, dt
     while total < budget_s:
         t0 = time.perf_counter()
-        cpu_oracle_step(wl, inp, list(range(n)), target[:n], oracle)
+        cpu_oracle_step(wl, inp, list(range(n)), target[:n], oracle, Whh)
         total += time.perf_counter() - t0
         reps += 1
     return {"value": reps * n * wl.gamma / total, "unit": UNIT, "cores": oracle.num_threads(),
@@ -300,6 +304,8 @@ def main():
     ap.add_argument("--eager", action="store_true", help="launch kernels one by one (no CUDA graph)")
     ap.add_argument("--stage", default="path", choices=["path", "sts-fit"],
                     help="path: the per-step hot path; sts-fit: the temperature fit")
+    ap.add_argument("--head", default="markov", choices=["markov", "rnn"],
+                    help="sequential block: Markov head, or RNN head (Elman reading)")
     ap.add_argument("--schedule", default="sync", choices=["sync", "lagged"],
                     help="sync: schedule on this step's scores; lagged: on the scores of two "
                          "steps earlier, on a side stream that overlaps the draft kernel")
@@ -344,6 +350,14 @@ def main():
         return torch.from_numpy(a).view(torch.bfloat16).cuda()
 
     U, h, W1, W2, w = bf(Uh), bf(hh), bf(W1h), bf(W2h), bf(wh)
+    rnn = args.head == "rnn"
+    Whh = bf(synth.whh(wl)) if rnn else None
+
+    def draft(**kw):
+        if rnn:
+            ds.draft_step_rnn(U, anchor, W1, W2, Whh, x, lx, ws, **kw)
+        else:
+            ds.draft_step(U, anchor, W1, W2, x, lx, ws, **kw)
     anchor = torch.from_numpy(anchor_h).cuda()
     T = torch.from_numpy(Th).cuda()
     Tstep = torch.from_numpy(Tstep_h).cuda()
@@ -362,8 +376,7 @@ def main():
     stream = torch.cuda.current_stream()
 
     # target tokens: the target model agrees with the drafts w.p. q_k (from a first draft)
-    ds.draft_step(U, anchor, W1, W2, x, lx, ws, mode=wl.mode, temperature=wl.tau, seed=wl.seed,
-                  b_offset=b0)
+    draft(mode=wl.mode, temperature=wl.tau, seed=wl.seed, b_offset=b0)
     torch.cuda.synchronize()
     target_h = synth.targets(wlg, x.cpu().numpy(), bs)
     target = torch.from_numpy(target_h).cuda()
@@ -385,8 +398,7 @@ def main():
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        ds.draft_step(U, anchor, W1, W2, x, lx, ws, mode=wl.mode, temperature=wl.tau,
-                      seed=wl.seed, b_offset=b0)
+        draft(mode=wl.mode, temperature=wl.tau, seed=wl.seed, b_offset=b0)
         if record is not None:
             e1.record(stream)
             record.append((e0, e1))
@@ -539,7 +551,8 @@ def main():
         t_tc = flops / (tflops * 1e12)
         roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "achieved": achieved,
                 "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
-                "traffic": _traffic_per_launch(wl.name), "kernel": "markov_draft_kernel",
+                "traffic": None if rnn else _traffic_per_launch(wl.name),
+                "kernel": "markov_draft_kernel",
                 "kernel_ms": draft_mean, "algorithmic_bytes": algo_bytes,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s"}
@@ -547,7 +560,8 @@ def main():
         if world == 1:
             inp = synth.Inputs(wl=wl, W1=W1h, W2=W2h, U=Uh, h=hh, anchor=anchor_h, w=wh, T=Th,
                                Tstep=Tstep_h, b_conf=wl.b_conf)
-            cpu = cpu_baseline(wl, inp, target_h, args.cpu_budget)
+            cpu = cpu_baseline(wl, inp, target_h, args.cpu_budget,
+                               synth.whh(wl) if rnn else None)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -563,6 +577,7 @@ def main():
             "gpu_launches": 4 * args.steps,
             "cuda_graph": graph is not None,
             "schedule": "lagged by 2 steps, side stream" if lagged else "this step's scores",
+            "head": args.head,
             "clocks": clk,
             "draft_kernel_ms": {"mean": draft_mean, "min": min(draft_ms), "max": max(draft_ms)},
         }

@@ -89,6 +89,25 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
                       void *workspace, size_t workspace_bytes, dspark_stream_t stream);
 
 /*
+ * RNN-head drafting: the second sequential block of [G] section 4 ("Two
+ * instantiations of the sequential block": a recurrent state that accumulates the
+ * block's prefix).  The pages give no equations; this is the Elman reading over the
+ * Markov head's factors:
+ *   s_0 = 0,  s_k = tanh(W1[x_{k-1}] + s_{k-1} Whh)     (fp32 state, r = 256)
+ *   l_k(v) = U[b, k-1, v] + sum_j bf16(s_k)[j] W2[j, v]
+ * and x_k, logit_x_out as in dspark_draft_step (greedy or Gumbel-max).
+ *   Whh [r, r] bf16 (row i, column j: s_{k-1}[i] contributes Whh[i][j] to element j),
+ *   16-byte aligned.  Every other argument as for dspark_draft_step; the workspace
+ *   from dspark_workspace_bytes also holds the [B, r] state.
+ * Cost over the Markov head: one more grid barrier per position and B r^2 MACs.
+ */
+int dspark_draft_step_rnn(const void *U, const int32_t *anchor, const void *W1, const void *W2,
+                          const void *Whh, int B, int gamma, int V, int r, int mode,
+                          float temperature, uint64_t seed, int b_offset, int32_t *x_out,
+                          float *logit_x_out, void *workspace, size_t workspace_bytes,
+                          dspark_stream_t stream);
+
+/*
  * Confidence head with Sequential Temperature Scaling and prefix survival.
  * [G] section 5 "Confidence-Scheduled Verification" (linear projection then
  * sigmoid over the backbone hidden state at position k and the Markov embedding

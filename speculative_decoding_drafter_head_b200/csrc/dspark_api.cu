@@ -81,7 +81,16 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 //                     schedule: ranks [n] i32, then fixed-point scores [n] i64
 constexpr size_t kCtlBytes = 256;
 
-size_t draft_ws(int B, int gamma) { return kCtlBytes + static_cast<size_t>(B) * gamma * 8; }
+//   RNN head: after the keys, the recurrent state [B][r] fp32 and its bf16 copy [B][r]
+size_t draft_keys_end(int B, int gamma)
+{
+    return round_up(kCtlBytes + static_cast<size_t>(B) * gamma * 8, 256);
+}
+
+size_t draft_ws(int B, int gamma)
+{
+    return draft_keys_end(B, gamma) + static_cast<size_t>(B) * 256 * (4 + 2);
+}
 
 size_t sched_ws(int n)
 {
@@ -146,14 +155,20 @@ int dspark_debug_barrier_extra(int extra)
     return DSPARK_OK;
 }
 
-int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, const void *W2, int B,
-                      int gamma, int V, int r, int mode, float temperature, uint64_t seed,
-                      int b_offset, int32_t *x_out, float *logit_x_out, void *workspace,
-                      size_t workspace_bytes, dspark_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// The Markov head (Whh == nullptr) and the RNN head share one kernel and one launcher.
+int launch_draft(const void *U, const int32_t *anchor, const void *W1, const void *W2,
+                 const void *Whh, int B, int gamma, int V, int r, int mode, float temperature,
+                 uint64_t seed, int b_offset, int32_t *x_out, float *logit_x_out, void *workspace,
+                 size_t workspace_bytes, dspark_stream_t stream)
 {
     namespace D = dspark::draft;
     if (!U || !anchor || !W1 || !W2 || !x_out || !logit_x_out || !workspace)
         return DSPARK_INVALID_ARG;
+    if (Whh && !aligned(Whh, 16)) return DSPARK_INVALID_ARG;
     if (!aligned(U, 16) || !aligned(W1, 16) || !aligned(W2, 16) || !aligned(anchor, 4) ||
         !aligned(x_out, 4) || !aligned(logit_x_out, 4) || !aligned(workspace, 256))
         return DSPARK_INVALID_ARG;
@@ -225,6 +240,10 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     prm.barrier = reinterpret_cast<unsigned int *>(ws);
     prm.abort_flag = reinterpret_cast<unsigned int *>(ws + 4);
     prm.slots = reinterpret_cast<unsigned long long *>(ws + kCtlBytes);
+    prm.Whh = static_cast<const uint16_t *>(Whh);
+    prm.state = reinterpret_cast<float *>(ws + draft_keys_end(B, gamma));
+    prm.a_rows = reinterpret_cast<uint16_t *>(ws + draft_keys_end(B, gamma) +
+                                              static_cast<size_t>(B) * 256 * 4);
     prm.units_total = (V + D::kUnit - 1) / D::kUnit;
     prm.M = M;
     prm.w2_stages = M == 64 ? 4 : 3;
@@ -235,7 +254,8 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     prm.timeout_ns = g_timeout_ns.load();
     prm.barrier_extra = g_barrier_extra.load();
 
-    if (cudaMemsetAsync(ws, 0, draft_ws(B, gamma), stream) != cudaSuccess) return DSPARK_CUDA_ERROR;
+    if (cudaMemsetAsync(ws, 0, draft_keys_end(B, gamma), stream) != cudaSuccess)
+        return DSPARK_CUDA_ERROR;
 
     const int grid = prm.units_total < dev->sms ? prm.units_total : dev->sms;
     cudaLaunchConfig_t cfg;
@@ -252,6 +272,30 @@ int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, cons
     if (M == 64)
         return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64>, tm_w2, tm_u, prm));
     return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128>, tm_w2, tm_u, prm));
+}
+
+}  // namespace
+
+extern "C" {
+
+int dspark_draft_step(const void *U, const int32_t *anchor, const void *W1, const void *W2, int B,
+                      int gamma, int V, int r, int mode, float temperature, uint64_t seed,
+                      int b_offset, int32_t *x_out, float *logit_x_out, void *workspace,
+                      size_t workspace_bytes, dspark_stream_t stream)
+{
+    return launch_draft(U, anchor, W1, W2, nullptr, B, gamma, V, r, mode, temperature, seed,
+                        b_offset, x_out, logit_x_out, workspace, workspace_bytes, stream);
+}
+
+int dspark_draft_step_rnn(const void *U, const int32_t *anchor, const void *W1, const void *W2,
+                          const void *Whh, int B, int gamma, int V, int r, int mode,
+                          float temperature, uint64_t seed, int b_offset, int32_t *x_out,
+                          float *logit_x_out, void *workspace, size_t workspace_bytes,
+                          dspark_stream_t stream)
+{
+    if (!Whh) return DSPARK_INVALID_ARG;
+    return launch_draft(U, anchor, W1, W2, Whh, B, gamma, V, r, mode, temperature, seed,
+                        b_offset, x_out, logit_x_out, workspace, workspace_bytes, stream);
 }
 
 int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x, const void *W1,

@@ -30,6 +30,7 @@
 // MMA uses M = 64 (rows 16q..16q+15 sit in TMEM lanes 32q..32q+15), else M = 128.
 #pragma once
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -81,6 +82,10 @@ struct Params {
     int u_slot_bytes;
     unsigned long long timeout_ns;
     int barrier_extra;
+    // RNN head (Whh != nullptr): s_k = tanh(W1[x_{k-1}] + s_{k-1} Whh), A_k = bf16(s_k)
+    const uint16_t *Whh;         // [r][r] bf16
+    float *state;                // [B][r] fp32, s_{k-1} then s_k (workspace)
+    uint16_t *a_rows;            // [B][r] bf16 copy of s_k, the rows the gather reads
 };
 
 struct Ctl {
@@ -703,10 +708,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int tok = __shfl_sync(0xFFFFFFFFu, my_tok, src_lane);
                 const int r = q * rq + src_lane;
                 const uint32_t dst = sA + chunk * a_chunk + r * 128 + ((unit ^ (r & 7)) << 4);
-                if (tok >= 0)
-                    cp_async_16(dst, p.W1 + static_cast<size_t>(tok) * kRank + lane * 8);
-                else
+                if (tok >= 0) {
+                    const uint16_t *src = p.Whh
+                        ? p.a_rows + static_cast<size_t>(gmt * M + r) * kRank    // row b of s_k
+                        : p.W1 + static_cast<size_t>(tok) * kRank;              // W1[x_{k-1}]
+                    cp_async_16(dst, src + lane * 8);
+                } else {
                     sts128_zero(dst);
+                }
             }
             cp_async_wait_all();
             fence_proxy_async_smem();
@@ -715,10 +724,95 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++mt_count;
         };
 
+        // bounded grid barrier number nth (counted from 1 over the whole launch); false
+        // once this CTA or any other gave up.  trace_k > 0 stamps the trace of position k.
+        auto grid_sync = [&](uint32_t nth, int trace_k) -> bool {
+            epi_sync();
+            if (threadIdx.x == 0 && ok && !*reinterpret_cast<volatile int *>(&ctl.abort)) {
+                red_release_add_u32(p.barrier, 1u);
+                if (trace_k > 0) DSPARK_TRACE_AT(trace_k, 4);
+                const uint32_t target =
+                    nth * static_cast<uint32_t>(G) + static_cast<uint32_t>(p.barrier_extra);
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_u32(p.barrier) < target) {
+                    if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
+                        *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
+                        break;
+                    }
+                    if (globaltimer_ns() - t0 > p.timeout_ns) {
+                        give_up(ctl, p, DSPARK_TIMEOUT);
+                        break;
+                    }
+                }
+                if (trace_k > 0) DSPARK_TRACE_AT(trace_k, 5);
+            }
+            epi_sync();
+            return ok && !*reinterpret_cast<volatile int *>(&ctl.abort);
+        };
+        const uint32_t bars_per_pos = p.Whh ? 2u : 1u;
+
+        // RNN head: this CTA's rows b = blockIdx.x + j G get s_k = tanh(W1[x_{k-1}] +
+        // s_{k-1} Whh).  Warp w multiplies Whh rows 32w .. 32w + 31 (16-byte loads, lane l
+        // holds columns 8l .. 8l + 7), the eight partial rows are summed through shared
+        // memory, and thread t finishes element t.  The A tile's shared memory, free until
+        // the gather that follows, holds s_{k-1} and the partial sums.
+        auto rnn_update = [&](int k) {
+            float *scr = reinterpret_cast<float *>(dyn_smem + (sA - smem_u32(dyn_smem)));
+            float *s_prev = scr;                          // [256]
+            float *part = scr + kRank;                    // [8][256]
+            const int t = threadIdx.x, w = t >> 5, ln = t & 31;
+            for (int b = blockIdx.x; b < p.B; b += G) {
+                int tok = k == 1 ? p.anchor[b]
+                                 : static_cast<int>(argmax_key_index(
+                                       __ldcg(&p.slots[static_cast<size_t>(k - 2) * p.B + b])));
+                tok = checked_token(tok, p.V);
+                float *st = p.state + static_cast<size_t>(b) * kRank;
+                s_prev[t] = k == 1 ? 0.0f : __ldcg(st + t);
+                epi_sync();
+                float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int ii = 0; ii < 32; ++ii) {
+                    const int i = 32 * w + ii;
+                    const float si = s_prev[i];
+                    const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(
+                        p.Whh + static_cast<size_t>(i) * kRank + 8 * ln));
+                    acc8[0] = fmaf(si, bf16lo_to_f32(wv.x), acc8[0]);
+                    acc8[1] = fmaf(si, bf16hi_to_f32(wv.x), acc8[1]);
+                    acc8[2] = fmaf(si, bf16lo_to_f32(wv.y), acc8[2]);
+                    acc8[3] = fmaf(si, bf16hi_to_f32(wv.y), acc8[3]);
+                    acc8[4] = fmaf(si, bf16lo_to_f32(wv.z), acc8[4]);
+                    acc8[5] = fmaf(si, bf16hi_to_f32(wv.z), acc8[5]);
+                    acc8[6] = fmaf(si, bf16lo_to_f32(wv.w), acc8[6]);
+                    acc8[7] = fmaf(si, bf16hi_to_f32(wv.w), acc8[7]);
+                }
+                float4 *pw = reinterpret_cast<float4 *>(part + w * kRank + 8 * ln);
+                pw[0] = make_float4(acc8[0], acc8[1], acc8[2], acc8[3]);
+                pw[1] = make_float4(acc8[4], acc8[5], acc8[6], acc8[7]);
+                epi_sync();
+                float acc = __uint_as_float(
+                    static_cast<uint32_t>(p.W1[static_cast<size_t>(tok) * kRank + t]) << 16);
+#pragma unroll
+                for (int q8 = 0; q8 < kEpiWarps; ++q8) acc += part[q8 * kRank + t];
+                const float sn = tanhf(acc);
+                st[t] = sn;
+                p.a_rows[static_cast<size_t>(b) * kRank + t] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(sn));
+                epi_sync();                   // the scratch is rewritten for the next row
+            }
+            __threadfence();                  // the rows are read by every CTA after the barrier
+        };
+
         for (int k = 1; k <= p.gamma && ok; ++k) {
             if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
                 ok = false;
                 break;
+            }
+            if (p.Whh) {
+                rnn_update(k);
+                if (!grid_sync(static_cast<uint32_t>(2 * k - 1), 0)) {
+                    ok = false;
+                    break;
+                }
             }
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 0);
             gather(0);
@@ -835,27 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // ---- grid barrier: every CTA has combined its rows of position k
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 3);
-            epi_sync();
-            if (threadIdx.x == 0 && ok && !*reinterpret_cast<volatile int *>(&ctl.abort)) {
-                red_release_add_u32(p.barrier, 1u);
-                DSPARK_TRACE_AT(k, 4);
-                const uint32_t target = static_cast<uint32_t>(k) * static_cast<uint32_t>(G) +
-                                        static_cast<uint32_t>(p.barrier_extra);
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_u32(p.barrier) < target) {
-                    if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
-                        *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
-                        break;
-                    }
-                    if (globaltimer_ns() - t0 > p.timeout_ns) {
-                        give_up(ctl, p, DSPARK_TIMEOUT);
-                        break;
-                    }
-                }
-                DSPARK_TRACE_AT(k, 5);
-            }
-            epi_sync();
-            if (!ok || *reinterpret_cast<volatile int *>(&ctl.abort)) {
+            if (!grid_sync(static_cast<uint32_t>(k) * bars_per_pos, k)) {
                 ok = false;
                 break;
             }

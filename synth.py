@@ -30,7 +30,7 @@ import numpy as np
 
 # stream tags (one per tensor kind)
 TAG_W1, TAG_W2, TAG_U, TAG_H, TAG_ANCHOR, TAG_W, TAG_T, TAG_TARGET, TAG_ZIPF = range(1, 10)
-TAG_SCORES, TAG_VERIFY, TAG_TSTEP, TAG_CALIB = 10, 11, 12, 13
+TAG_SCORES, TAG_VERIFY, TAG_TSTEP, TAG_CALIB, TAG_WHH = 10, 11, 12, 13, 14
 
 _THREADS = max(1, min(16, os.cpu_count() or 1))
 
@@ -133,6 +133,12 @@ def w1(wl: Workload) -> np.ndarray:
 def w2(wl: Workload) -> np.ndarray:
     """Markov logits projection W2 [r, V] (bf16 bits), N(0, w_std^2)."""
     return _normal_bf16(_rng(wl.seed, TAG_W2), wl.r * wl.V, wl.w_std).reshape(wl.r, wl.V)
+
+
+def whh(wl: Workload, std: float = 0.04) -> np.ndarray:
+    """RNN-head recurrence Whh [r, r] (bf16 bits), N(0, std^2); 0.04 sqrt(256) = 0.64 keeps
+    the recurrence contractive under tanh."""
+    return _normal_bf16(_rng(wl.seed, TAG_WHH), wl.r * wl.r, std).reshape(wl.r, wl.r)
 
 
 def anchors(wl: Workload) -> np.ndarray:

@@ -113,3 +113,15 @@ def test_sts_fit_host_checks():
     assert call(N=0) == 2 and call(N=1 << 23) == 2     # fixed-point sums need N < 2^23
     assert call(gamma=65) == 2 and call(n_bins=257) == 2 and call(n_t=0) == 2
     assert call(wsb=need - 1) == 3
+
+
+def test_draft_step_rnn_host_checks():
+    lib = ds.load()
+    f = _FAKE
+    # a null or misaligned recurrence matrix is rejected before anything is enqueued
+    assert lib.dspark_draft_step_rnn(f, f, f, f, None, 4, 2, 4096, 256, 0, 1.0, 0, 0, f, f, f,
+                                     1 << 20, None) == 1
+    assert lib.dspark_draft_step_rnn(f, f, f, f, C.c_void_p(0x10008), 4, 2, 4096, 256, 0, 1.0, 0,
+                                     0, f, f, f, 1 << 20, None) == 1
+    # the workspace also holds the [B, 256] state: fp32 + bf16 per row
+    assert ds.workspace_bytes(1000, 16, 4096) >= 1000 * 256 * 6
