@@ -213,10 +213,16 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     }
 
     if (!dev->draft_attr_set) {
-        if (cudaFuncSetAttribute(D::markov_draft_kernel<64>,
+        if (cudaFuncSetAttribute(D::markov_draft_kernel<64, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  D::kDynSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(D::markov_draft_kernel<128>,
+            cudaFuncSetAttribute(D::markov_draft_kernel<128, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 D::kDynSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(D::markov_draft_kernel<64, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 D::kDynSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(D::markov_draft_kernel<128, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  D::kDynSmem) != cudaSuccess)
             return DSPARK_CUDA_ERROR;
@@ -269,9 +275,15 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (M == 64)
-        return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64>, tm_w2, tm_u, prm));
-    return from_cuda(cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128>, tm_w2, tm_u, prm));
+    cudaError_t e;
+    if (Whh)
+        e = M == 64 ? cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64, true>, tm_w2, tm_u, prm)
+                    : cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128, true>, tm_w2, tm_u, prm);
+    else
+        e = M == 64 ? cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64, false>, tm_w2, tm_u, prm)
+                    : cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128, false>, tm_w2, tm_u,
+                                         prm);
+    return from_cuda(e);
 }
 
 }  // namespace

@@ -459,8 +459,9 @@ __device__ __forceinline__ void box_update_m64(RowBest (&best)[2], const uint32_
     }
 }
 
-// kM is the MMA's M (64 when B <= 64, else 128); p.M equals it.
-template <int kM>
+// kM is the MMA's M (64 when B <= 64, else 128); p.M equals it.  kRnn selects the RNN
+// head (p.Whh set); the Markov instances carry none of its code.
+template <int kM, bool kRnn>
 __global__ void __launch_bounds__(kThreads, 1)
     markov_draft_kernel(const __grid_constant__ CUtensorMap tm_w2,
                         const __grid_constant__ CUtensorMap tm_u, const Params p)
@@ -709,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int r = q * rq + src_lane;
                 const uint32_t dst = sA + chunk * a_chunk + r * 128 + ((unit ^ (r & 7)) << 4);
                 if (tok >= 0) {
-                    const uint16_t *src = p.Whh
+                    const uint16_t *src = kRnn
                         ? p.a_rows + static_cast<size_t>(gmt * M + r) * kRank    // row b of s_k
                         : p.W1 + static_cast<size_t>(tok) * kRank;              // W1[x_{k-1}]
                     cp_async_16(dst, src + lane * 8);
@@ -749,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             epi_sync();
             return ok && !*reinterpret_cast<volatile int *>(&ctl.abort);
         };
-        const uint32_t bars_per_pos = p.Whh ? 2u : 1u;
+        constexpr uint32_t bars_per_pos = kRnn ? 2u : 1u;
 
         // RNN head: this CTA's rows b = blockIdx.x + j G get s_k = tanh(W1[x_{k-1}] +
         // s_{k-1} Whh).  Warp w multiplies Whh rows 32w .. 32w + 31 (16-byte loads, lane l
@@ -807,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            if (p.Whh) {
+            if constexpr (kRnn) {
                 rnn_update(k);
                 if (!grid_sync(static_cast<uint32_t>(2 * k - 1), 0)) {
                     ok = false;

@@ -182,6 +182,10 @@ STRESS = [
     synth.Workload("stress B=33 V=9000 gumbel", B=33, gamma=4, V=9000, d=64, w_std=0.2,
                    logits="normal", mode=1, tau=0.9, seed=3),
     synth.Workload("stress B=64 V=4104", B=64, gamma=5, V=4104, d=64, w_std=0.2, seed=2),
+    # 5 and 10 units (160 and 320 columns) per CTA: a one-unit remainder tile on every CTA
+    synth.Workload("stress B=20 V=23680", B=20, gamma=4, V=23680, d=64, w_std=0.2, seed=7),
+    synth.Workload("stress B=48 V=47360 gumbel", B=48, gamma=3, V=47360, d=64, w_std=0.2,
+                   mode=1, tau=0.8, seed=8),
     # the largest gamma the kernel takes, one row and a 130-row tile pair
     synth.Workload("stress B=3 gamma=64 V=2048", B=3, gamma=64, V=2048, d=64, w_std=0.3, seed=4),
     synth.Workload("stress B=130 gamma=64 V=1032", B=130, gamma=64, V=1032, d=64, w_std=0.3,
