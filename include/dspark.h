@@ -112,7 +112,7 @@ int dspark_draft_step_rnn(const void *U, const int32_t *anchor, const void *W1, 
  * [G] section 5 "Confidence-Scheduled Verification" (linear projection then
  * sigmoid over the backbone hidden state at position k and the Markov embedding
  * of the previous draft token; temperature scaling per position) and [S]
- * ("per-position prefix survival probabilities", a cumulative product).
+ * (the survival probability of every prefix of the block, a cumulative product).
  *
  *   z_{b,k} = sum_i w[i] h[b, k-1, i] + sum_j w[d + j] W1[x_{k-1}, j] + b_conf
  *   c_{b,k} = 1 / (1 + exp(-z_{b,k} / T[k-1]))
@@ -135,7 +135,8 @@ int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x
  * Hardware-aware prefix scheduler: per-request verify lengths that maximise
  * expected accepted tokens per unit time.
  * [W] "The Hardware-Aware Prefix Scheduler" (throughput maximisation against a
- * steps-per-second curve) and [G] section 6 ("global throughput maximization").
+ * steps-per-second curve) and [G] section 6 (the choice is posed as maximising the
+ * throughput of the whole batch).
  *
  * Scores P[b, k-1] (non-increasing in k, within [0, 1]) are ordered by
  * (P desc, b asc, k asc); q = floor(P 2^46); S_N = sum of the first N q's;

@@ -31,8 +31,8 @@
  *   - confidence: c_k = sigmoid(z_k / T_k) with
  *     z_k = w . [h_k ; W1[x_{k-1}]] + b  ([G] section 5, "Sequential
  *     Temperature Scaling" applied to the whole logit);
- *   - prefix survival: P_k = prod_{j <= k} c_j  ([W], [S]: "prefix survival
- *     probabilities", [G] section 5: "cumulative product");
+ *   - prefix survival: P_k = prod_{j <= k} c_j  ([W], [S]: the survival probability
+ *     of each prefix; [G] section 5: a cumulative product);
  *   - scheduler objective: expected tokens per second
  *     F = (B + sum_b sum_{k <= L_b} P_{b,k}) / Tstep(B + sum_b L_b), scores
  *     fixed-point q = floor(P 2^46), order (P desc, b asc, k asc), first
@@ -354,7 +354,7 @@ int oracle_confidence(const uint16_t *h, const int32_t *anchor, const int32_t *x
 
 /* --------------------------------------------------------------------------
  * Hardware-aware prefix scheduler ([W] "The Hardware-Aware Prefix Scheduler";
- * [G] section 6, "global throughput maximization").
+ * [G] section 6, the batch-wide throughput maximisation).
  *
  * Scores P[b, k-1] (fp32) are ordered by (P desc, b asc, k asc).  With
  * q = floor(P 2^46) (exact integers) and S_N the sum of the first N of them,
