@@ -122,9 +122,10 @@ int dspark_draft_step_rnn(const void *U, const int32_t *anchor, const void *W1, 
  *   h [B, gamma, d] bf16;  anchor [B] int32;  x [B, gamma] int32 (last column unused)
  *   W1 [V, r] bf16;  w [d + r] bf16;  T [gamma] fp32 (> 0)
  *   c_out, P_out [B, gamma] fp32
- * Supported sizes: 1 <= B, 1 <= gamma <= 64, d % 8 == 0, r % 8 == 0; h, W1, w
- * 16-byte aligned.  A token id outside [0, V) records DSPARK_INVALID_TOKEN and is
- * read as 0.
+ * Supported sizes: 1 <= B <= 65535, 1 <= gamma <= 64, d % 8 == 0, r % 8 == 0,
+ * (d + r) 2 <= 200 KB; h, W1, w 16-byte aligned.  A token id outside [0, V) records
+ * DSPARK_INVALID_TOKEN and is read as 0.  Launched as one thread-block cluster of up to
+ * 8 CTAs per request.
  */
 int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x,
                           const void *W1, const void *w, float b_conf, const float *T,

@@ -319,20 +319,29 @@ int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x
     if (!aligned(h, 16) || !aligned(W1, 16) || !aligned(w, 16) || !aligned(anchor, 4) ||
         !aligned(x, 4) || !aligned(T, 4) || !aligned(c_out, 4) || !aligned(P_out, 4))
         return DSPARK_INVALID_ARG;
-    if (B < 1 || gamma < 1 || gamma > C::kMaxGamma || d < 8 || d % 8 != 0 || r < 8 ||
+    if (B < 1 || B > 65535 || gamma < 1 || gamma > C::kMaxGamma || d < 8 || d % 8 != 0 || r < 8 ||
         r % 8 != 0 || V < 1 || (d + r) * 2 > 200 * 1024)
         return DSPARK_UNSUPPORTED_SHAPE;
     DeviceInfo *dev = nullptr;
     if (int st = current_device(&dev)) return st;
-    const int smem = (d + r) * 2;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(C::confidence_sts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-        return DSPARK_CUDA_ERROR;
-    C::confidence_sts_kernel<<<B, C::kThreads, smem, stream>>>(
-        static_cast<const uint16_t *>(h), anchor, x, static_cast<const uint16_t *>(W1),
-        static_cast<const uint16_t *>(w), b_conf, T, B, gamma, d, r, V, c_out, P_out);
-    return from_cuda(cudaGetLastError());
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    const int cs = C::cluster_ctas(gamma);
+    cfg.gridDim = dim3(cs, B);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return from_cuda(cudaLaunchKernelEx(
+        &cfg, C::confidence_sts_kernel, static_cast<const uint16_t *>(h), anchor, x,
+        static_cast<const uint16_t *>(W1), static_cast<const uint16_t *>(w), b_conf, T, B, gamma,
+        d, r, V, c_out, P_out));
 }
 
 int dspark_schedule_prefix(const float *P, int B, int gamma, const double *Tstep_us,
