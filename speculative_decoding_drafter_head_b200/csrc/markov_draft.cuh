@@ -1,33 +1,37 @@
-// markov_draft.cuh -- the sequential Markov head of DSpark on tcgen05 tensor cores.
+// markov_draft.cuh -- the sequential head of DSpark (Markov or RNN) on tcgen05 tensor cores.
 //
 // gdymind.com, "DSpark: DeepSeek's new speculative decoding work", section 4
 // ("Sequential stage", "Markov head"): position k adds a first-order transition
 // bias B(x_{k-1}, .) = W1[x_{k-1}] W2 (rank r = 256) to the backbone's base logits
-// U_k and picks x_k from them.
+// U_k and picks x_k from them.  The same section names an RNN head, a recurrent state
+// over the block's prefix; with kRnn the bias is bf16(s_k) W2 instead, where
+// s_k = tanh(W1[x_{k-1}] + s_{k-1} Whh) (our reading; the pages give no equations).
 //
 // One persistent cooperative kernel runs all gamma positions.  Each CTA owns a
 // contiguous slice of the vocabulary (a whole number of 32-column units, balanced
-// over the grid) cut into tiles of up to 256 columns, and for every position k and
-// every block of M requests it computes
-//     D[b, v] = sum_j A[b, j] W2[j, v],   A[b, :] = W1[x_{k-1, b}, :]
+// over the grid) cut into tiles of 128 columns, and for every position k and every
+// block of M requests it computes
+//     D[b, v] = sum_j A[b, j] W2[j, v],   A[b, :] = W1[x_{k-1, b}, :]  (or bf16(s_k[b, :]))
 // as tcgen05.mma M=64/128, N<=128, K=16 (bf16 in, fp32 accumulate in TMEM), with W2
 // streamed by TMA in two K-halves of 128 rows (MN-major, 128-byte swizzle).  A single
 // MMA instruction costs the same for any N up to 128 and for M = 64 or 128, so tiles
-// are 128 columns wide and a CTA's odd remainder becomes one narrow tile.  The
-// epilogue adds U_k (staged by TMA), applies greedy or Gumbel-max selection and keeps
-// a running (max, index) per request row, so the [B, V] logits never reach memory.
-// Rows are
+// are 128 columns wide and a CTA's remainder becomes one narrower tile.  The epilogue
+// adds U_k (staged by TMA), applies greedy or Gumbel-max selection and keeps a running
+// (max, index) per request row, so the [B, V] logits never reach memory.  Rows are
 // combined across CTAs by a 64-bit atomicMax on (ordered value, inverted index); a
 // bounded grid barrier ends each position, after which every CTA reads x_k for the
-// next gather and the CTA that owns the winning column writes the outputs.
+// next gather and the CTA that owns the winning column writes the outputs.  The RNN
+// instance adds, before each gather, the state update of the CTA's rows and a second
+// grid barrier that publishes them.
 //
 // W2 is read with an L2 evict-last policy and U with evict-first: within one launch
 // W2 (at most 134 MB) is re-read every position and mostly stays in L2.
 //
 // Warp roles (352 threads): warps 0-7 epilogue and A gather (warps q and q + 4 read
-// TMEM lane quadrant q and split each tile's 32-column chunks between them), warp 8
-// W2 producer, warp 9 U producer, warp 10 MMA issuer and TMEM owner.  With B <= 64 the
-// MMA uses M = 64 (rows 16q..16q+15 sit in TMEM lanes 32q..32q+15), else M = 128.
+// TMEM lane quadrant q and take alternate 64-column boxes of each tile), warp 8 W2
+// producer, warp 9 U producer, warp 10 MMA issuer and TMEM owner.  With B <= 64 the MMA
+// uses M = 64 (rows 16q..16q+15 sit in TMEM lanes 32q..32q+15, read with 16x256b loads),
+// else M = 128 (32x32b loads).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
