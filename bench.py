@@ -53,8 +53,15 @@ def _peaks():
 
 
 def _kernel_sha():
-    with open(DRAFT_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the draft kernel's source with comments and blank space removed, so that the
+    committed DRAM-traffic figure stays attached to the code it was measured on."""
+    import re
+    with open(DRAFT_SRC, encoding="utf-8") as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = re.sub(r"\s+", " ", src).strip()
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
 def _traffic_per_launch(workload_name):
