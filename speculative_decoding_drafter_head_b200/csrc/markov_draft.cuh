@@ -347,11 +347,11 @@ __device__ __forceinline__ void box_update(RowBest &best, const uint32_t (&a0)[3
         if (m0 == mx) {
             const int idx = first_index(s0, mx);
             best.v = static_cast<uint32_t>(v0 + idx);
-            best.l = pick(l0, idx);
+            best.l = p.mode == 0 ? mx : pick(l0, idx);     // greedy: the score is the logit
         } else {
             const int idx = first_index(s1, mx);
             best.v = static_cast<uint32_t>(v0 + kUnit + idx);
-            best.l = pick(l1, idx);
+            best.l = p.mode == 0 ? mx : pick(l1, idx);
         }
         best.s = mx;
     }
@@ -452,10 +452,12 @@ __device__ __forceinline__ void box_update_m64(RowBest (&best)[2], const uint32_
 #pragma unroll
                 for (int e = 1; e >= 0; --e)
                     if (s[4 * i + 2 * h + e] == mx) idx = 4 * i + 2 * h + e;
-            float li = l[2 * h];
+            float li = mx;                      // greedy: the score is the logit
+            if (p.mode != 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (j == idx) li = l[j];
+                for (int j = 0; j < 32; ++j)
+                    if (j == idx) li = l[j];
+            }
             best[h].v = static_cast<uint32_t>(vw + 8 * (idx >> 2) + (idx & 1));
             best[h].l = li;
             best[h].s = mx;
