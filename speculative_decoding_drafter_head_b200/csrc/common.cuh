@@ -42,6 +42,20 @@ __device__ unsigned long long g_trace[256 * 64 * 32];
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Two fp32 additions in one packed instruction (add.rn.f32x2): d0 = a0 + b0, d1 = a1 + b1,
+// each rounded to nearest as a plain fp32 addition would be.
+__device__ __forceinline__ void add_f32x2(float &d0, float &d1, float a0, float a1, float b0,
+                                          float b1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ float warp_sum(float v)
 {
 #pragma unroll

@@ -260,14 +260,14 @@ __device__ __forceinline__ void add_u32(float (&l)[32], const uint32_t (&a)[32],
     for (int u = 0; u < 4; ++u) {
         uint32_t w0, w1, w2, w3;
         lds128(sU + row * 128 + (((4 * h + u) ^ (row & 7)) << 4), w0, w1, w2, w3);
-        l[8 * u + 0] = __uint_as_float(a[8 * u + 0]) + bf16lo_to_f32(w0);
-        l[8 * u + 1] = __uint_as_float(a[8 * u + 1]) + bf16hi_to_f32(w0);
-        l[8 * u + 2] = __uint_as_float(a[8 * u + 2]) + bf16lo_to_f32(w1);
-        l[8 * u + 3] = __uint_as_float(a[8 * u + 3]) + bf16hi_to_f32(w1);
-        l[8 * u + 4] = __uint_as_float(a[8 * u + 4]) + bf16lo_to_f32(w2);
-        l[8 * u + 5] = __uint_as_float(a[8 * u + 5]) + bf16hi_to_f32(w2);
-        l[8 * u + 6] = __uint_as_float(a[8 * u + 6]) + bf16lo_to_f32(w3);
-        l[8 * u + 7] = __uint_as_float(a[8 * u + 7]) + bf16hi_to_f32(w3);
+        add_f32x2(l[8 * u + 0], l[8 * u + 1], __uint_as_float(a[8 * u + 0]),
+                  __uint_as_float(a[8 * u + 1]), bf16lo_to_f32(w0), bf16hi_to_f32(w0));
+        add_f32x2(l[8 * u + 2], l[8 * u + 3], __uint_as_float(a[8 * u + 2]),
+                  __uint_as_float(a[8 * u + 3]), bf16lo_to_f32(w1), bf16hi_to_f32(w1));
+        add_f32x2(l[8 * u + 4], l[8 * u + 5], __uint_as_float(a[8 * u + 4]),
+                  __uint_as_float(a[8 * u + 5]), bf16lo_to_f32(w2), bf16hi_to_f32(w2));
+        add_f32x2(l[8 * u + 6], l[8 * u + 7], __uint_as_float(a[8 * u + 6]),
+                  __uint_as_float(a[8 * u + 7]), bf16lo_to_f32(w3), bf16hi_to_f32(w3));
     }
 }
 
@@ -380,10 +380,10 @@ __device__ __forceinline__ void box_update_m64(RowBest (&best)[2], const uint32_
     for (int i = 0; i < 8; ++i) {
         const uint32_t wa = lds32(sU + ua * 128 + ((i ^ (ua & 7)) << 4) + w * 4);
         const uint32_t wb = lds32(sU + ub * 128 + ((i ^ (ub & 7)) << 4) + w * 4);
-        l[4 * i + 0] = __uint_as_float(a[4 * i + 0]) + bf16lo_to_f32(wa);
-        l[4 * i + 1] = __uint_as_float(a[4 * i + 1]) + bf16hi_to_f32(wa);
-        l[4 * i + 2] = __uint_as_float(a[4 * i + 2]) + bf16lo_to_f32(wb);
-        l[4 * i + 3] = __uint_as_float(a[4 * i + 3]) + bf16hi_to_f32(wb);
+        add_f32x2(l[4 * i + 0], l[4 * i + 1], __uint_as_float(a[4 * i + 0]),
+                  __uint_as_float(a[4 * i + 1]), bf16lo_to_f32(wa), bf16hi_to_f32(wa));
+        add_f32x2(l[4 * i + 2], l[4 * i + 3], __uint_as_float(a[4 * i + 2]),
+                  __uint_as_float(a[4 * i + 3]), bf16lo_to_f32(wb), bf16hi_to_f32(wb));
     }
     const int vw = v0 + 2 * w;                    // column of a[0]
     if (!two || v0 + 2 * kUnit > p.V) {
