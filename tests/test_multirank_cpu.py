@@ -75,3 +75,19 @@ def test_noise_keys_use_global_request_index(oracle_mod):
     shard, _, _ = oracle_mod.draft(U[3:], anchor[3:], W1, W2, mode=1, tau=0.8, seed=5,
                                    b_index=np.arange(3, B, dtype=np.int32))
     np.testing.assert_array_equal(shard, full[3:])
+
+
+def test_rnn_noise_keys_use_global_request_index(oracle_mod):
+    """The RNN head drafted on a shard with its global request ids equals the same rows of
+    the full batch (the state is per request, so sharding by request keeps it local)."""
+    V, r, gamma, B = 300, 8, 4, 6
+    rng = np.random.default_rng(3)
+    U = synth.f32_to_bf16_bits(rng.normal(0, 1, (B, gamma, V)).astype(np.float32))
+    W1 = synth.f32_to_bf16_bits(rng.normal(0, 0.3, (V, r)).astype(np.float32))
+    W2 = synth.f32_to_bf16_bits(rng.normal(0, 0.3, (r, V)).astype(np.float32))
+    Whh = synth.f32_to_bf16_bits(rng.normal(0, 0.2, (r, r)).astype(np.float32))
+    anchor = rng.integers(0, V, B).astype(np.int32)
+    full, _, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh, mode=1, tau=0.8, seed=5)
+    shard, _, _ = oracle_mod.draft_rnn(U[2:], anchor[2:], W1, W2, Whh, mode=1, tau=0.8, seed=5,
+                                       b_index=np.arange(2, B, dtype=np.int32))
+    np.testing.assert_array_equal(shard, full[2:])

@@ -534,3 +534,21 @@ def test_rnn_rejects_bad_anchor(oracle_mod):
     anchor[1] = 50
     with pytest.raises(ValueError):
         oracle_mod.draft_rnn(U, anchor, W1, W2, Whh)
+
+
+def test_rnn_without_projection_drafts_the_backbone_argmax(oracle_mod):
+    # W2 = 0: no bias at all, whatever the state; the draft is the argmax of U per position
+    V, r, gamma, nb = 200, 8, 5, 3
+    U, anchor, W1, W2, Whh = _rnn_inputs(nb, gamma, V, r, 12, 0.5)
+    x, l, _ = oracle_mod.draft_rnn(U, anchor, W1, np.zeros_like(W2), Whh)
+    np.testing.assert_array_equal(x, np.argmax(_f(U), axis=2))
+    np.testing.assert_array_equal(l, np.max(_f(U), axis=2))
+
+
+def test_rnn_gumbel_at_low_temperature_is_greedy(oracle_mod):
+    # tau -> 0: l / tau dominates the bounded noise, so Gumbel-max selects the argmax
+    V, r, gamma, nb = 300, 8, 4, 3
+    U, anchor, W1, W2, Whh = _rnn_inputs(nb, gamma, V, r, 13, 0.3)
+    xg, _, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh)
+    xs, _, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh, mode=1, tau=1e-6, seed=4)
+    np.testing.assert_array_equal(xs, xg)
