@@ -44,10 +44,10 @@ def _load():
         lib.oracle_gumbel.argtypes = [C.c_uint64, C.c_int, C.c_int, C.c_int]
         lib.oracle_gumbel.restype = C.c_double
         lib.oracle_draft.argtypes = [p, p, p, p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
-                                     C.c_double, C.c_uint64, p, p, p, p, C.c_int]
+                                     C.c_double, C.c_uint64, p, p, p, p, p, C.c_int]
         lib.oracle_draft.restype = C.c_int
         lib.oracle_draft_rnn.argtypes = [p, p, p, p, p, C.c_int, C.c_int, C.c_int, C.c_int,
-                                         C.c_int, C.c_double, C.c_uint64, p, p, p, p, C.c_int]
+                                         C.c_int, C.c_double, C.c_uint64, p, p, p, p, p, C.c_int]
         lib.oracle_draft_rnn.restype = C.c_int
         lib.oracle_confidence.argtypes = [p, p, p, p, p, C.c_double, p, C.c_int, C.c_int,
                                           C.c_int, C.c_int, C.c_int, p, p, p, p, C.c_int]
@@ -93,9 +93,21 @@ def gumbel(seed: int, b: int, k: int, v: int) -> float:
     return float(_load().oracle_gumbel(int(seed), int(b), int(k), int(v)))
 
 
+def _forced(forced_prev, nb, gamma):
+    if forced_prev is None:
+        return None, None
+    fp = _c(forced_prev, np.int32)
+    assert fp.shape == (nb, gamma)
+    return fp, _ptr(fp)
+
+
 def draft(U, anchor, W1, W2, mode: int = 0, tau: float = 1.0, seed: int = 0, b_index=None,
-          nthreads: int = 0):
-    """Markov-head drafting; returns (x [nb, gamma] int32, logit [nb, gamma] f64, gap f64)."""
+          nthreads: int = 0, forced_prev=None):
+    """Markov-head drafting; returns (x [nb, gamma] int32, logit [nb, gamma] f64, gap f64).
+
+    forced_prev [nb, gamma] (optional): teacher-forced use, position k conditions on
+    x_{k-1} = forced_prev[:, k-1] rather than on the token this call picked at k - 1.
+    """
     U = _c(U, np.uint16)
     nb, gamma, V = U.shape
     W1 = _c(W1, np.uint16)
@@ -108,16 +120,17 @@ def draft(U, anchor, W1, W2, mode: int = 0, tau: float = 1.0, seed: int = 0, b_i
     x = np.zeros((nb, gamma), dtype=np.int32)
     logit = np.zeros((nb, gamma), dtype=np.float64)
     gap = np.zeros((nb, gamma), dtype=np.float64)
+    fp, fp_ptr = _forced(forced_prev, nb, gamma)
     st = _load().oracle_draft(_ptr(U), _ptr(anchor), _ptr(W1), _ptr(W2), nb, gamma, V, r,
                               int(mode), float(tau), int(seed) & (2**64 - 1), _ptr(bi), _ptr(x),
-                              _ptr(logit), _ptr(gap), int(nthreads))
+                              _ptr(logit), _ptr(gap), fp_ptr, int(nthreads))
     if st != 0:
         raise ValueError(f"oracle_draft rejected its arguments (status {st})")
     return x, logit, gap
 
 
 def draft_rnn(U, anchor, W1, W2, Whh, mode: int = 0, tau: float = 1.0, seed: int = 0,
-              b_index=None, nthreads: int = 0):
+              b_index=None, nthreads: int = 0, forced_prev=None):
     """RNN-head drafting (Elman reading); returns (x, logit, gap) as draft()."""
     U = _c(U, np.uint16)
     nb, gamma, V = U.shape
@@ -131,9 +144,11 @@ def draft_rnn(U, anchor, W1, W2, Whh, mode: int = 0, tau: float = 1.0, seed: int
     x = np.zeros((nb, gamma), dtype=np.int32)
     logit = np.zeros((nb, gamma), dtype=np.float64)
     gap = np.zeros((nb, gamma), dtype=np.float64)
+    fp, fp_ptr = _forced(forced_prev, nb, gamma)
     st = _load().oracle_draft_rnn(_ptr(U), _ptr(anchor), _ptr(W1), _ptr(W2), _ptr(Whh), nb,
                                   gamma, V, r, int(mode), float(tau), int(seed) & (2**64 - 1),
-                                  _ptr(bi), _ptr(x), _ptr(logit), _ptr(gap), int(nthreads))
+                                  _ptr(bi), _ptr(x), _ptr(logit), _ptr(gap), fp_ptr,
+                                  int(nthreads))
     if st != 0:
         raise ValueError(f"oracle_draft_rnn rejected its arguments (status {st})")
     return x, logit, gap

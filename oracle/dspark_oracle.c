@@ -122,11 +122,16 @@ double oracle_gumbel(uint64_t seed, int b, int k, int v)
  *   x_k      = smallest v with s(v) = max s
  *   logit[k] = l(x_k);  gap[k] = max s - second largest s (0 on an exact tie)
  * with x_0 = anchor[i].  U holds only the listed requests: [nb, gamma, V].
+ *
+ * Teacher-forced use (forced_prev non-NULL, [nb, gamma]): position k conditions on
+ * x_{k-1} = forced_prev[i, k-1] instead of the token this call picked at k - 1, so
+ * every position is the one-step Markov transition from a given previous token (the
+ * same arithmetic; only where x_{k-1} comes from differs).
  * ------------------------------------------------------------------------ */
 int oracle_draft(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
                  const uint16_t *W2, int nb, int gamma, int V, int r, int mode, double tau,
                  uint64_t seed, const int32_t *b_index, int32_t *x_out, double *logit_out,
-                 double *gap_out, int nthreads)
+                 double *gap_out, const int32_t *forced_prev, int nthreads)
 {
     if (nb < 0 || gamma < 1 || V < 2 || r < 1 || (mode != 0 && mode != 1))
         return ORACLE_INVALID;
@@ -135,6 +140,10 @@ int oracle_draft(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
     for (int i = 0; i < nb; ++i)
         if (anchor[i] < 0 || anchor[i] >= V)
             return ORACLE_INVALID;
+    if (forced_prev)
+        for (size_t o = 0; o < (size_t)nb * (size_t)gamma; ++o)
+            if (forced_prev[o] < 0 || forced_prev[o] >= V)
+                return ORACLE_INVALID;
     if (nthreads < 1)
         nthreads = oracle_num_threads();
 
@@ -149,6 +158,8 @@ int oracle_draft(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
         }
         int prev = anchor[i];
         for (int k = 1; k <= gamma; ++k) {
+            if (forced_prev)
+                prev = forced_prev[(size_t)i * (size_t)gamma + (size_t)(k - 1)];
             const uint16_t *row = W1 + (size_t)prev * (size_t)r;
             for (int v = 0; v < V; ++v)
                 bias[v] = 0.0;
@@ -198,6 +209,8 @@ int oracle_draft(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
  *   l_k(v) = U[b, k-1, v] + sum_j a_k[j] W2[j, v]
  * and x_k is chosen as in oracle_draft (greedy or Gumbel-max).  With Whh = 0
  * the bias is that of a Markov head whose table is bf16(fp32(tanh(W1))).
+ * forced_prev (optional, [nb, gamma]) gives x_{k-1} for every position as in
+ * oracle_draft; the state then runs along the given tokens.
  * ------------------------------------------------------------------------ */
 static uint16_t f32_to_bf16_rne(float f)
 {
@@ -212,7 +225,8 @@ static uint16_t f32_to_bf16_rne(float f)
 int oracle_draft_rnn(const uint16_t *U, const int32_t *anchor, const uint16_t *W1,
                      const uint16_t *W2, const uint16_t *Whh, int nb, int gamma, int V, int r,
                      int mode, double tau, uint64_t seed, const int32_t *b_index,
-                     int32_t *x_out, double *logit_out, double *gap_out, int nthreads)
+                     int32_t *x_out, double *logit_out, double *gap_out,
+                     const int32_t *forced_prev, int nthreads)
 {
     if (nb < 0 || gamma < 1 || V < 2 || r < 1 || (mode != 0 && mode != 1))
         return ORACLE_INVALID;
@@ -221,6 +235,10 @@ int oracle_draft_rnn(const uint16_t *U, const int32_t *anchor, const uint16_t *W
     for (int i = 0; i < nb; ++i)
         if (anchor[i] < 0 || anchor[i] >= V)
             return ORACLE_INVALID;
+    if (forced_prev)
+        for (size_t o = 0; o < (size_t)nb * (size_t)gamma; ++o)
+            if (forced_prev[o] < 0 || forced_prev[o] >= V)
+                return ORACLE_INVALID;
     if (nthreads < 1)
         nthreads = oracle_num_threads();
 
@@ -240,6 +258,8 @@ int oracle_draft_rnn(const uint16_t *U, const int32_t *anchor, const uint16_t *W
         }
         int prev = anchor[i];
         for (int k = 1; k <= gamma; ++k) {
+            if (forced_prev)
+                prev = forced_prev[(size_t)i * (size_t)gamma + (size_t)(k - 1)];
             const uint16_t *row = W1 + (size_t)prev * (size_t)r;
             for (int j = 0; j < r; ++j) {
                 double acc = bf16_to_f64(row[j]);

@@ -292,13 +292,14 @@ def targets(wl: Workload, drafts: np.ndarray, bs: Optional[Sequence[int]] = None
 # inputs for the scheduler and verify stages on their own
 # ----------------------------------------------------------------------------
 def monotone_scores(B: int, gamma: int, seed: int, tie_frac: float = 0.0,
-                    zero_frac: float = 0.0) -> np.ndarray:
+                    zero_frac: float = 0.0, neg_zero: bool = False) -> np.ndarray:
     """Scores P [B, gamma] (fp32) in [0, 1] that never increase along a row.
 
     Values are uniform draws sorted in decreasing order within each row.  With
     tie_frac > 0 some entries repeat their left neighbour and some values are
     copied across rows, so that equal scores occur within and across requests;
-    zero_frac sets a tail of some rows to exactly 0.
+    zero_frac sets a tail of some rows to exactly 0; with neg_zero, about half of
+    those zeros are written as -0.0 (equal to +0.0 as a number, sign bit set).
     """
     rng = _rng(seed, TAG_SCORES, B, gamma)
     P = np.sort(rng.random((B, gamma)).astype(np.float32), axis=1)[:, ::-1].copy()
@@ -318,6 +319,9 @@ def monotone_scores(B: int, gamma: int, seed: int, tie_frac: float = 0.0,
             if rng.random() < zero_frac:
                 cut = int(rng.integers(0, gamma + 1))
                 P[b, cut:] = 0.0
+        if neg_zero:
+            flip = (P == 0.0) & (rng.random((B, gamma)) < 0.5)
+            P[flip] = np.float32(-0.0)
     return np.ascontiguousarray(P, dtype=np.float32)
 
 

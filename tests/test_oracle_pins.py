@@ -87,6 +87,42 @@ def test_draft_rejects_bad_anchor(oracle_mod):
         oracle_mod.draft(U, np.array([64], np.int32), W1, W2)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_draft_forced_on_its_own_tokens_is_the_free_running_draft(oracle_mod, mode):
+    # teacher forcing with x_{k-1} = the tokens the free-running draft picked must give
+    # back that draft exactly (greedy and Gumbel-max, whose noise is keyed by position)
+    V, r, gamma, nb = 400, 16, 7, 5
+    U, anchor, W1, W2 = _tiny_draft_inputs(nb, gamma, V, r, 0.4, seed=21)
+    x, l, g = oracle_mod.draft(U, anchor, W1, W2, mode=mode, tau=0.8, seed=5)
+    prev = np.concatenate([anchor[:, None], x[:, :-1]], axis=1)
+    xf, lf, gf = oracle_mod.draft(U, anchor, W1, W2, mode=mode, tau=0.8, seed=5, forced_prev=prev)
+    np.testing.assert_array_equal(xf, x)
+    np.testing.assert_array_equal(lf, l)
+    np.testing.assert_array_equal(gf, g)
+
+
+def test_draft_forced_position_is_a_one_step_draft_from_that_token(oracle_mod):
+    # greedy: position k forced to x_{k-1} = t equals a one-position draft whose anchor
+    # is t and whose base logits are U[:, k-1] (catches an off-by-one in the forcing)
+    V, r, gamma, nb = 300, 16, 6, 4
+    U, anchor, W1, W2 = _tiny_draft_inputs(nb, gamma, V, r, 0.5, seed=22)
+    prev = np.random.default_rng(3).integers(0, V, (nb, gamma)).astype(np.int32)
+    xf, lf, gf = oracle_mod.draft(U, anchor, W1, W2, forced_prev=prev)
+    for k in range(gamma):
+        x1, l1, g1 = oracle_mod.draft(U[:, k:k + 1].copy(), prev[:, k].copy(), W1, W2)
+        np.testing.assert_array_equal(xf[:, k], x1[:, 0])
+        np.testing.assert_array_equal(lf[:, k], l1[:, 0])
+        np.testing.assert_array_equal(gf[:, k], g1[:, 0])
+
+
+def test_draft_forced_rejects_out_of_range_tokens(oracle_mod):
+    U, anchor, W1, W2 = _tiny_draft_inputs(2, 3, 64, 8, 0.1, seed=1)
+    prev = np.zeros((2, 3), np.int32)
+    prev[1, 2] = 64
+    with pytest.raises(ValueError):
+        oracle_mod.draft(U, anchor, W1, W2, forced_prev=prev)
+
+
 # ---------------------------------------------------------------------------
 # Gumbel-max: frequencies must follow softmax(l / tau)
 # ---------------------------------------------------------------------------
@@ -332,6 +368,22 @@ def test_schedule_worked_examples_of_the_pages(oracle_mod):
         np.testing.assert_allclose(F_all[:len(case["F_by_N"])], case["F_by_N"], rtol=2e-4)
 
 
+def test_schedule_negative_zero_scores_count_as_zero(oracle_mod):
+    # -0.0 equals +0.0 as a number: the same lengths, N* and objective as with +0.0,
+    # and exact zeros keep their (b asc, k asc) order behind every positive score
+    B, gamma = 24, 6
+    rng = np.random.default_rng(8)
+    P = synth.monotone_scores(B, gamma, seed=2, tie_frac=0.2, zero_frac=0.6, neg_zero=True)
+    assert np.signbit(P).any()
+    Pp = np.where(P == 0.0, np.float32(0.0), P).astype(np.float32)
+    for Tstep in _tables(B, gamma, rng):
+        a = oracle_mod.schedule(P, Tstep)
+        b = oracle_mod.schedule(Pp, Tstep)
+        np.testing.assert_array_equal(a[0], b[0])
+        assert a[1] == b[1] and a[2] == b[2]
+        np.testing.assert_array_equal(a[3], b[3])
+
+
 def test_schedule_rejects_scores_outside_unit_interval(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.schedule(np.array([[1.5, 0.5]], np.float32), np.ones(4))
@@ -552,3 +604,45 @@ def test_rnn_gumbel_at_low_temperature_is_greedy(oracle_mod):
     xg, _, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh)
     xs, _, _ = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh, mode=1, tau=1e-6, seed=4)
     np.testing.assert_array_equal(xs, xg)
+
+
+def test_rnn_recurrence_is_row_vector_times_whh(oracle_mod):
+    # Hand-computed two-position case that fixes the orientation of the recurrence,
+    # s_k[j] = tanh(W1[x_{k-1}][j] + sum_q s_{k-1}[q] Whh[q][j]).  Whh has one entry,
+    # Whh[1][2] = a; W2 is the identity on the first r tokens, so the bias at token
+    # v < r is bf16(s_k[v]).
+    #   position 1: s_1 = tanh(W1[anchor]) = (0, tanh 1, 0, 0); U forces x_1 = 10.
+    #   position 2: W1[10] = 0, so s_2 = tanh(s_1 Whh) = (0, 0, tanh(a tanh 1), 0) and
+    #   U = 0 on tokens < r (-100 elsewhere): x_2 = 2 with logit bf16(tanh(a tanh 1)).
+    # The transposed reading (Whh s) would give s_2 = tanh(a s_1[2]) e_1 = 0, x_2 = 0.
+    V, r, a = 64, 4, 0.5
+    W1 = np.zeros((V, r), np.float32)
+    anchor_tok = 20
+    W1[anchor_tok, 1] = 1.0
+    W2 = np.zeros((r, V), np.float32)
+    W2[np.arange(r), np.arange(r)] = 1.0
+    Whh = np.zeros((r, r), np.float32)
+    Whh[1, 2] = a
+    Uf = np.full((1, 2, V), -100.0, np.float32)
+    Uf[0, 0, 10] = 50.0
+    Uf[0, 1, :r] = 0.0
+    x, l, g = oracle_mod.draft_rnn(_bf16(Uf), np.array([anchor_tok], np.int32), _bf16(W1),
+                                   _bf16(W2), _bf16(Whh))
+    s2 = math.tanh(a * math.tanh(1.0))
+    expect = float(_f(_bf16([s2]))[0])
+    assert x[0, 0] == 10 and l[0, 0] == 50.0
+    assert x[0, 1] == 2
+    assert l[0, 1] == expect
+    assert g[0, 1] == expect          # every other token of the first r has logit 0
+
+
+def test_rnn_forced_on_its_own_tokens_is_the_free_running_draft(oracle_mod):
+    V, r, gamma, nb = 300, 8, 6, 3
+    U, anchor, W1, W2, Whh = _rnn_inputs(nb, gamma, V, r, 14, 0.4)
+    x, l, g = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh, mode=1, tau=0.9, seed=2)
+    prev = np.concatenate([anchor[:, None], x[:, :-1]], axis=1)
+    xf, lf, gf = oracle_mod.draft_rnn(U, anchor, W1, W2, Whh, mode=1, tau=0.9, seed=2,
+                                      forced_prev=prev)
+    np.testing.assert_array_equal(xf, x)
+    np.testing.assert_array_equal(lf, l)
+    np.testing.assert_array_equal(gf, g)
