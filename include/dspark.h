@@ -230,9 +230,12 @@ int dspark_sts_fit(const float *z, const int32_t *accepted, int N, int gamma, do
  *     contents: calls that can overlap on the GPU (different streams, or different host
  *     threads without ordering between their streams) race and give wrong results;
  *     order them on one stream;
- *   - the first call on each device looks the array's device address up
- *     (cudaGetSymbolAddress) with that device current; make that first call before any
- *     stream capture.
+ *   - every call looks the array's device address up (cudaGetSymbolAddress) with the
+ *     calling device current.  The first call on a device may make the CUDA runtime
+ *     load this library's device code there (lazy module loading), which allocates
+ *     device memory for the image and can synchronise the device: make that first call
+ *     during start-up, before any stream capture.  From the second call on, the call
+ *     neither allocates nor synchronises.
  */
 int dspark_schedule_prefix_noalloc(const float *P, int B, int gamma, const double *Tstep_us,
                                    int32_t *L_out, int32_t *N_out, double *objective_out,

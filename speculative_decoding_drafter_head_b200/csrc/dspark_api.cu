@@ -45,7 +45,6 @@ EncodeTiledFn encode_tiled()
 struct DeviceInfo {
     int sms = 0;
     int major = 0;
-    bool draft_attr_set = false;
 };
 
 constexpr int kMaxDevices = 64;
@@ -212,22 +211,14 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
             return DSPARK_CUDA_ERROR;
     }
 
-    if (!dev->draft_attr_set) {
-        if (cudaFuncSetAttribute(D::markov_draft_kernel<64, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 D::kDynSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(D::markov_draft_kernel<128, false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 D::kDynSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(D::markov_draft_kernel<64, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 D::kDynSmem) != cudaSuccess ||
-            cudaFuncSetAttribute(D::markov_draft_kernel<128, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 D::kDynSmem) != cudaSuccess)
-            return DSPARK_CUDA_ERROR;
-        dev->draft_attr_set = true;
-    }
+    // the kernel instance for this call (Markov or RNN head, M = 64 or 128); its shared
+    // memory limit is set on every call, so nothing cached outlives a device reset
+    void (*kern)(const CUtensorMap, const CUtensorMap, const D::Params) =
+        Whh ? (M == 64 ? D::markov_draft_kernel<64, true> : D::markov_draft_kernel<128, true>)
+            : (M == 64 ? D::markov_draft_kernel<64, false> : D::markov_draft_kernel<128, false>);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::kDynSmem) !=
+        cudaSuccess)
+        return DSPARK_CUDA_ERROR;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     D::Params prm;
@@ -275,15 +266,7 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e;
-    if (Whh)
-        e = M == 64 ? cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64, true>, tm_w2, tm_u, prm)
-                    : cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128, true>, tm_w2, tm_u, prm);
-    else
-        e = M == 64 ? cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<64, false>, tm_w2, tm_u, prm)
-                    : cudaLaunchKernelEx(&cfg, D::markov_draft_kernel<128, false>, tm_w2, tm_u,
-                                         prm);
-    return from_cuda(e);
+    return from_cuda(cudaLaunchKernelEx(&cfg, kern, tm_w2, tm_u, prm));
 }
 
 }  // namespace
@@ -491,11 +474,6 @@ constexpr size_t kNoAllocScratchBytes = kNoAllocQOffset + static_cast<size_t>(kN
 
 static __device__ __align__(256) unsigned char g_sched_scratch[kNoAllocScratchBytes];
 
-// Device address of g_sched_scratch per device (0 until that device's first call).
-// In host code the symbol names only a host-side stand-in, so the address is looked up
-// with cudaGetSymbolAddress while the device is current.
-void *g_sched_scratch_dev[kMaxDevices];
-
 }  // namespace
 
 extern "C" {
@@ -514,19 +492,12 @@ int dspark_schedule_prefix_noalloc(const float *P, int B, int gamma, const doubl
         return DSPARK_UNSUPPORTED_SHAPE;
     DeviceInfo *dev = nullptr;
     if (int st = current_device(&dev)) return st;
-    int dev_id = 0;
-    if (cudaGetDevice(&dev_id) != cudaSuccess) return DSPARK_CUDA_ERROR;
+    // In host code g_sched_scratch names only a host-side stand-in; its device address
+    // on the current device is looked up on every call (cheap once the module is
+    // loaded), so no address outlives a context that was torn down and re-created.
     void *scratch = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(g_dev_mutex);
-        if (!g_sched_scratch_dev[dev_id]) {
-            void *addr = nullptr;
-            if (cudaGetSymbolAddress(&addr, g_sched_scratch) != cudaSuccess || !addr)
-                return DSPARK_CUDA_ERROR;
-            g_sched_scratch_dev[dev_id] = addr;
-        }
-        scratch = g_sched_scratch_dev[dev_id];
-    }
+    if (cudaGetSymbolAddress(&scratch, g_sched_scratch) != cudaSuccess || !scratch)
+        return DSPARK_CUDA_ERROR;
     uint8_t *ws = static_cast<uint8_t *>(scratch);
     const int n = B * gamma;
     S::Params prm;

@@ -36,6 +36,11 @@ struct Params {
     unsigned int *done;     // completion counter, zeroed before launch
 };
 
+// Bits of a score for ordering.  Valid scores lie in [0, 1], where the fp32 bit
+// patterns of non-negative values sort like the values, once -0.0 (sign bit set, equal
+// to +0.0 as a number) is mapped onto +0.0 by adding +0.0.
+__device__ __forceinline__ uint32_t score_bits(float p) { return __float_as_uint(p + 0.0f); }
+
 // Number of entries of row `row` ordered before the score (bits pb, flat index ib).
 __device__ __forceinline__ int count_before(const float *__restrict__ P, int gamma, int row,
                                             uint32_t pb, int ib)
@@ -44,7 +49,7 @@ __device__ __forceinline__ int count_before(const float *__restrict__ P, int gam
     int lo = 0, hi = gamma;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        const uint32_t m = __float_as_uint(__ldg(pr + mid));
+        const uint32_t m = score_bits(__ldg(pr + mid));
         const bool before = (m > pb) || (m == pb && row * gamma + mid < ib);
         if (before)
             lo = mid + 1;
@@ -92,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params 
     // ---------------- phase 1: ranks
     for (int i = blockIdx.x * kWarps + warp; i < p.n; i += gridDim.x * kWarps) {
         const float pi = __ldg(p.P + i);
-        const uint32_t pb = __float_as_uint(pi);
+        const uint32_t pb = score_bits(pi);
         int cnt = 0;
         for (int row = lane; row < p.B; row += 32) cnt += count_before(p.P, p.gamma, row, pb, i);
 #pragma unroll

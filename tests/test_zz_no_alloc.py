@@ -35,7 +35,7 @@ def _schedule(lib, fn_name, P, Tstep, ws=None):
     return L.cpu().numpy(), int(N.item()), float(F.item())
 
 
-def test_noalloc_scheduler_matches_workspace_scheduler_on_consecutive_calls():
+def test_noalloc_scheduler_matches_workspace_scheduler_on_consecutive_calls(oracle_mod):
     import torch
     import speculative_decoding_drafter_head_b200 as ds
     lib = ds.load()
@@ -43,16 +43,23 @@ def test_noalloc_scheduler_matches_workspace_scheduler_on_consecutive_calls():
     f.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                   C.c_void_p]
     f.restype = C.c_int
-    cases = [(64, 16, 0.0), (1024, 24, 0.3)]          # two calls in a row, different sizes
-    for B, gamma, tie in cases:
-        P = synth.monotone_scores(B, gamma, seed=B, tie_frac=tie)
+    # calls in a row that share the static scratch: the largest size first, so that a
+    # smaller call runs over leftovers of a larger one; then a case with -0.0 scores
+    # (equal to +0.0) and ties, and the largest size again
+    cases = [(1024, 24, 0.3, 0.0, False), (64, 16, 0.0, 0.0, False),
+             (512, 16, 0.2, 0.5, True), (1024, 24, 0.0, 0.0, False)]
+    for B, gamma, tie, zero, negz in cases:
+        P = synth.monotone_scores(B, gamma, seed=B, tie_frac=tie, zero_frac=zero, neg_zero=negz)
         n = np.arange(B * (gamma + 1) + 1, dtype=np.float64)
         Tstep = 15000.0 + 20.0 * np.maximum(0.0, n - (B * (gamma + 1)) // 3)
         ws = torch.empty(ds.workspace_bytes(B, gamma, 1000), dtype=torch.uint8, device="cuda")
         ref = _schedule(lib, "dspark_schedule_prefix", P, Tstep, ws)
         got = _schedule(lib, "dspark_schedule_prefix_noalloc", P, Tstep)
+        L_or, N_or, F_or, _ = oracle_mod.schedule(P, Tstep)
         np.testing.assert_array_equal(got[0], ref[0])
         assert got[1] == ref[1] and got[2] == ref[2]
+        np.testing.assert_array_equal(got[0], L_or)
+        assert got[1] == N_or and got[2] == F_or
         assert 0 < ref[1] <= B * gamma
     assert ds.get_error() == 0
 
