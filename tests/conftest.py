@@ -18,3 +18,18 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Draft parity of the session: positions compared, oracle near ties, mismatches."""
+    try:
+        from helpers import PARITY_LOG
+    except Exception:
+        return
+    if not PARITY_LOG:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "draft parity (every position, oracle teacher-forced on the GPU's tokens)")
+    for name, c in PARITY_LOG:
+        tr.write_line(f"{name}: compared {c.compared}, near ties {c.near_ties}, "
+                      f"hard mismatches {c.hard_mismatch}, max |logit err| {c.max_logit_err:.2e}")
