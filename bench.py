@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
+PARITY_MACS = 3.5e11          # oracle multiply-adds spent on the bench line's parity check
 METRIC = "draft tokens/s (Markov head+confidence+schedule+verify); % of HBM/TC roofline"
 UNIT = "tokens/s"
 DRAFT_SRC = os.path.join(ROOT, "speculative_decoding_drafter_head_b200", "csrc", "markov_draft.cuh")
@@ -132,6 +133,13 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_config(wl, world=1):
+    """The `config` object both arms print (identical keys and values)."""
+    return {"workload": wl.name, "B_per_gpu": wl.B, "gamma": wl.gamma, "V": wl.V, "r": wl.r,
+            "d": wl.d, "mode": "gumbel" if wl.mode else "greedy", "parallelism": f"dp{world}",
+            "l2_flush": True}
+
+
 def cpu_oracle_step(wl, inp, bs, target_rows, oracle, Whh=None):
     """The oracle's whole path on the listed requests (one bounded sample of a step)."""
     bs = list(bs)
@@ -177,8 +185,7 @@ def run_reference(args, wl):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sec / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "gamma": wl.gamma, "V": wl.V, "r": wl.r,
-                   "d": wl.d, "mode": "gumbel" if wl.mode else "greedy"},
+        "config": workload_config(wl, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{len(sample)} of {wl.B} requests per step, whole path"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -211,6 +218,49 @@ def cpu_baseline(wl, inp, target, budget_s, Whh=None):
     return {"value": reps * n * wl.gamma / total, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle", "sample": f"{n} of {wl.B} requests x {reps} full steps "
                                         f"(draft, confidence, schedule, verify), {total:.1f} s"}
+
+
+def parity_report(wl, inp, target, out, oracle, Whh=None, n_rows=None, schedule=True):
+    """The GPU outputs of one timed step against the oracle (outside every timed region).
+
+    Drafts: every position of the first n_rows requests against the oracle run
+    teacher-forced on the GPU's previous tokens; tokens may differ only where the oracle's
+    top-2 gap is below 2e-2 (near ties), the logit at a matching token within 2e-2.
+    Confidence: c and P against the oracle fed the GPU's drafts.  Scheduler and verify:
+    bit for bit against the oracle fed the GPU's scores and lengths.
+    """
+    tol = 2e-2
+    n = wl.B if n_rows is None else min(n_rows, wl.B)
+    bs = list(range(n))
+    x, lx = out["x"][:n], out["lx"][:n]
+    prev = np.concatenate([inp.anchor[:n, None], x[:, :-1]], axis=1).astype(np.int32)
+    U = synth.u_requests(wl, bs) if inp.U is None else inp.U[:n]
+    if Whh is None:
+        xo, lo, go = oracle.draft(U, inp.anchor[:n], inp.W1, inp.W2, mode=wl.mode, tau=wl.tau,
+                                  seed=wl.seed, b_index=np.array(bs, np.int32), forced_prev=prev)
+    else:
+        xo, lo, go = oracle.draft_rnn(U, inp.anchor[:n], inp.W1, inp.W2, Whh, mode=wl.mode,
+                                      tau=wl.tau, seed=wl.seed, b_index=np.array(bs, np.int32),
+                                      forced_prev=prev)
+    same = x == xo
+    rep = {"rows": n, "positions": int(x.size), "compared": int(same.sum()),
+           "near_ties": int((~same & (go < tol)).sum()),
+           "hard_mismatch": int((~same & (go >= tol)).sum()),
+           "max_logit_err": float(np.abs(lx[same] - lo[same]).max()) if same.any() else 0.0}
+    h = synth.h_requests(wl, bs) if inp.h is None else inp.h[:n]
+    conf = oracle.confidence(h, inp.anchor[:n], x, inp.W1, inp.w, inp.b_conf, inp.T)
+    rep["max_c_err"] = float(np.abs(out["c"][:n] - conf["c"]).max())
+    if schedule:            # the scores of this step fed this step's scheduler
+        rep["max_P_err"] = float(np.abs(out["P"][:n] - conf["P64"]).max())
+        L_or, N_or, F_or, _ = oracle.schedule(out["P"], inp.Tstep)
+        rep["schedule_bit_exact"] = bool((out["L"] == L_or).all() and out["N"] == N_or and
+                                         out["F"] == F_or)
+    a_or, b_or = oracle.verify(out["x"], out["L"], target)
+    rep["verify_bit_exact"] = bool((out["acc"] == a_or).all() and (out["bonus"] == b_or).all())
+    rep["ok"] = bool(rep["hard_mismatch"] == 0 and rep["max_logit_err"] <= tol and
+                     rep["max_c_err"] <= tol and rep.get("max_P_err", 0.0) <= tol and
+                     rep.get("schedule_bit_exact", True) and rep["verify_bit_exact"])
+    return rep
 
 
 STS_METRIC = "STS fit candidate evaluations/s (blocks x gamma x grid temperatures)"
@@ -488,6 +538,12 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     total_ms = sum(step_ms)
     assert ds.get_error() == 0, "device error during the timed steps"
+    # outputs of the last timed step, checked against the oracle after all timing
+    snap = None
+    if world == 1:
+        snap = {"x": x.cpu().numpy(), "lx": lx.cpu().numpy(), "c": c.cpu().numpy(),
+                "P": P.cpu().numpy(), "L": last_L[0].cpu().numpy(), "N": int(Nst.item()),
+                "F": float(obj.item()), "acc": acc.cpu().numpy(), "bonus": bonus.cpu().numpy()}
 
     # the draft kernel alone, for its roofline (same inputs, L2 flushed before each launch)
     for _ in range(args.steps):
@@ -563,22 +619,26 @@ def main():
                 "kernel_ms": draft_mean, "algorithmic_bytes": algo_bytes,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s"}
-        cpu = None
+        cpu = parity = None
         if world == 1:
             inp = synth.Inputs(wl=wl, W1=W1h, W2=W2h, U=Uh, h=hh, anchor=anchor_h, w=wh, T=Th,
                                Tstep=Tstep_h, b_conf=wl.b_conf)
-            cpu = cpu_baseline(wl, inp, target_h, args.cpu_budget,
-                               synth.whh(wl) if rnn else None)
+            Whh_h = synth.whh(wl) if rnn else None
+            cpu = cpu_baseline(wl, inp, target_h, args.cpu_budget, Whh_h)
+            import oracle
+            # every request when the oracle can redo the step in a few seconds, else the first
+            rows = max(1, min(B, int(PARITY_MACS / (gamma * wl.r * V))))
+            parity = parity_report(wl, inp, target_h, snap, oracle, Whh_h, n_rows=rows,
+                                   schedule=not lagged)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": wl.name, "B_per_gpu": B, "gamma": gamma, "V": V, "r": wl.r,
-                       "d": wl.d, "mode": "gumbel" if wl.mode else "greedy",
-                       "parallelism": f"dp{world}", "l2_flush": True},
+            "config": workload_config(wl, world),
             "roofline": roof,
             "cpu_baseline": cpu,
+            "parity": parity,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": 4 * args.steps,
@@ -586,7 +646,9 @@ def main():
             "schedule": "lagged by 2 steps, side stream" if lagged else "this step's scores",
             "head": args.head,
             "clocks": clk,
-            "draft_kernel_ms": {"mean": draft_mean, "min": min(draft_ms), "max": max(draft_ms)},
+            "ms_per_step_median": statistics.median(step_ms),
+            "draft_kernel_ms": {"mean": draft_mean, "median": statistics.median(draft_ms),
+                                "min": min(draft_ms), "max": max(draft_ms)},
         }
         print(json.dumps(line), flush=True)
     graph = None                                    # release the graphs before the group

@@ -25,3 +25,32 @@ def test_reference_arm_json_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert "workload" in d["config"]
+    import bench
+    import synth
+    assert d["config"] == bench.workload_config(synth.TINY, 1)   # same keys as the GPU arm
+
+
+def test_parity_report_counts_mismatches(oracle_mod):
+    """The bench line's parity summary, fed the oracle's own step, reports no mismatch; a
+    token changed at a position with a clear oracle margin counts as a hard mismatch."""
+    import numpy as np
+    import bench
+    import synth
+    wl = synth.TINY.with_(V=4000, d=64)
+    inp = synth.make_inputs(wl)
+    x, l, g = oracle_mod.draft(inp.U, inp.anchor, inp.W1, inp.W2)
+    conf = oracle_mod.confidence(inp.h, inp.anchor, x, inp.W1, inp.w, inp.b_conf, inp.T)
+    P = conf["P32"]
+    L, N, F, _ = oracle_mod.schedule(P, inp.Tstep)
+    target = synth.targets(wl, x)
+    acc, bonus = oracle_mod.verify(x, L, target)
+    out = {"x": x, "lx": l.astype(np.float32), "c": conf["c"].astype(np.float32), "P": P,
+           "L": L, "N": N, "F": F, "acc": acc, "bonus": bonus}
+    rep = bench.parity_report(wl, inp, target, out, oracle_mod)
+    assert rep["ok"] and rep["hard_mismatch"] == 0 and rep["compared"] == x.size
+    assert rep["schedule_bit_exact"] and rep["verify_bit_exact"]
+    b, k = np.argwhere(g > 0.1)[0]
+    bad = dict(out, x=x.copy())
+    bad["x"][b, k] = (x[b, k] + 1) % wl.V
+    rep = bench.parity_report(wl, inp, target, bad, oracle_mod, schedule=False)
+    assert not rep["ok"] and rep["hard_mismatch"] >= 1
