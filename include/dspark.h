@@ -133,6 +133,29 @@ int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x
                           dspark_stream_t stream);
 
 /*
+ * Drafting and the confidence head in one call: the results of dspark_draft_step
+ * followed by dspark_confidence_sts on the drafted tokens.
+ * [G] section 4 (Markov head) and section 5 (the confidence head reads the backbone
+ * hidden state at k and the Markov embedding of x_{k-1}, the row the draft gathers).
+ *
+ * Arguments as for those two calls (U, anchor, W1, W2, mode, temperature, seed, b_offset,
+ * x_out, logit_x_out, workspace as for dspark_draft_step; h, w, b_conf, T, d, c_out,
+ * P_out as for dspark_confidence_sts), with the same sizes, alignment and errors.  With
+ * B <= 128 both run in one launch: one warp of every CTA of the draft kernel computes
+ * the hidden-state part of every logit at the start and the rest of each position's
+ * scores as soon as the grid barrier of the previous position has fixed x_{k-1}, beside
+ * the drafting; the workspace from dspark_workspace_bytes covers it.  With B > 128 the
+ * confidence kernel follows as a second launch on the same stream.  c and P agree with
+ * dspark_confidence_sts up to the order of the fp32 additions of z.
+ */
+int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const void *W1,
+                                 const void *W2, const void *h, const void *w, float b_conf,
+                                 const float *T, int B, int gamma, int V, int r, int d, int mode,
+                                 float temperature, uint64_t seed, int b_offset, int32_t *x_out,
+                                 float *logit_x_out, float *c_out, float *P_out, void *workspace,
+                                 size_t workspace_bytes, dspark_stream_t stream);
+
+/*
  * Hardware-aware prefix scheduler: per-request verify lengths that maximise
  * expected accepted tokens per unit time.
  * [W] "The Hardware-Aware Prefix Scheduler" (throughput maximisation against a

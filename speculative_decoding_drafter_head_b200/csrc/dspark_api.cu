@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "confidence_sts.cuh"
 #include "markov_draft.cuh"
+#include "markov_pair.cuh"
 #include "ptx.cuh"
 #include "schedule_prefix.cuh"
 #include "sts_fit.cuh"
@@ -45,9 +46,11 @@ EncodeTiledFn encode_tiled()
 struct DeviceInfo {
     int sms = 0;
     int major = 0;
+    bool no_coop_clusters = false;   // the runtime refused a cooperative cluster launch
 };
 
 constexpr int kMaxDevices = 64;
+constexpr int kW2StagesM64 = 5;   // W2 ring depth of the M = 64 instance (32 KB stages)
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -158,11 +161,23 @@ int dspark_debug_barrier_extra(int extra)
 
 namespace {
 
-// The Markov head (Whh == nullptr) and the RNN head share one kernel and one launcher.
+// Inputs and outputs of the confidence head when it runs inside the draft launch.
+struct ConfArgs {
+    const void *h;
+    const void *w;
+    float b_conf;
+    const float *T;
+    int d;
+    float *c_out;
+    float *P_out;
+};
+
+// The Markov head (Whh == nullptr) and the RNN head share one kernel and one launcher;
+// with `conf` the Markov head's launch also computes the confidence head.
 int launch_draft(const void *U, const int32_t *anchor, const void *W1, const void *W2,
                  const void *Whh, int B, int gamma, int V, int r, int mode, float temperature,
                  uint64_t seed, int b_offset, int32_t *x_out, float *logit_x_out, void *workspace,
-                 size_t workspace_bytes, dspark_stream_t stream)
+                 size_t workspace_bytes, dspark_stream_t stream, const ConfArgs *conf = nullptr)
 {
     namespace D = dspark::draft;
     if (!U || !anchor || !W1 || !W2 || !x_out || !logit_x_out || !workspace)
@@ -183,6 +198,8 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     EncodeTiledFn encode = encode_tiled();
     if (!encode) return DSPARK_CUDA_ERROR;
 
+    // more than 128 requests (Markov head): the CTA-pair kernel, M = 256 per pair MMA
+    const bool pair = !Whh && B > 128;
     const int M = B <= 64 ? 64 : 128;
     const int ub = B < M ? B : M;
     CUtensorMap tm_w2, tm_u;
@@ -211,12 +228,18 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
             return DSPARK_CUDA_ERROR;
     }
 
-    // the kernel instance for this call (Markov or RNN head, M = 64 or 128); its shared
-    // memory limit is set on every call, so nothing cached outlives a device reset
+    // the kernel instance for this call (Markov or RNN head, M = 64 or 128, or the pair
+    // kernel); its shared memory limit is set on every call, so nothing cached outlives a
+    // device reset
+    const bool fused = conf && !pair;    // the pair kernel leaves confidence to its own launch
     void (*kern)(const CUtensorMap, const CUtensorMap, const D::Params) =
-        Whh ? (M == 64 ? D::markov_draft_kernel<64, true> : D::markov_draft_kernel<128, true>)
-            : (M == 64 ? D::markov_draft_kernel<64, false> : D::markov_draft_kernel<128, false>);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::kDynSmem) !=
+        pair ? D::pairk::markov_pair_kernel
+        : Whh ? (M == 64 ? D::markov_draft_kernel<64, true> : D::markov_draft_kernel<128, true>)
+        : fused ? (M == 64 ? D::markov_draft_kernel<64, false, true>
+                           : D::markov_draft_kernel<128, false, true>)
+                : (M == 64 ? D::markov_draft_kernel<64, false> : D::markov_draft_kernel<128, false>);
+    const int dyn_smem = pair ? D::pairk::kDynSmem : D::kDynSmem;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem) !=
         cudaSuccess)
         return DSPARK_CUDA_ERROR;
 
@@ -243,28 +266,77 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
                                               static_cast<size_t>(B) * 256 * 4);
     prm.units_total = (V + D::kUnit - 1) / D::kUnit;
     prm.M = M;
-    prm.w2_stages = M == 64 ? 4 : 3;
+    // shared memory: A (M x 256 bf16), then the W2 ring, then U boxes in what is left
+    prm.w2_stages = M == 64 ? kW2StagesM64 : 3;
     prm.ub = ub;
     prm.u_slot_bytes = static_cast<int>(round_up(static_cast<size_t>(ub) * D::kUBoxCols * 2, 1024));
-    prm.u_slots = D::kURingBytes / prm.u_slot_bytes;
+    prm.u_slots = (D::kRingSmem - M * D::kRank * 2 - prm.w2_stages * D::kW2StageBytes) /
+                  prm.u_slot_bytes;
     if (prm.u_slots > D::kUMaxSlots) prm.u_slots = D::kUMaxSlots;
     prm.timeout_ns = g_timeout_ns.load();
     prm.barrier_extra = g_barrier_extra.load();
+    if (fused) {
+        prm.h = static_cast<const uint16_t *>(conf->h);
+        prm.wconf = static_cast<const uint16_t *>(conf->w);
+        prm.b_conf = conf->b_conf;
+        prm.T = conf->T;
+        prm.d = conf->d;
+        prm.c_out = conf->c_out;
+        prm.P_out = conf->P_out;
+        prm.zh = reinterpret_cast<float *>(ws + draft_keys_end(B, gamma));   // the RNN state's space
+        prm.zh_done = reinterpret_cast<unsigned int *>(ws + 8);
+    }
 
     if (cudaMemsetAsync(ws, 0, draft_keys_end(B, gamma), stream) != cudaSuccess)
         return DSPARK_CUDA_ERROR;
 
-    const int grid = prm.units_total < dev->sms ? prm.units_total : dev->sms;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(D::kThreads);
-    cfg.dynamicSmemBytes = D::kDynSmem;
+    cfg.dynamicSmemBytes = dyn_smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
+    if (!pair) {
+        const int grid = prm.units_total < dev->sms ? prm.units_total : dev->sms;
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(fused ? D::kThreadsConf : D::kThreads);
+        cfg.numAttrs = 1;
+        return from_cuda(cudaLaunchKernelEx(&cfg, kern, tm_w2, tm_u, prm));
+    }
+    // clusters of two CTAs, as many pairs as can be resident at once (every CTA waits for
+    // all others at the end of each position)
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(D::pairk::kThreads);
+    cfg.gridDim = dim3(dev->sms & ~1);
+    cfg.attrs = attr + 1;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+        cudaGetLastError();
+        return DSPARK_CUDA_ERROR;
+    }
+    int npairs = dev->sms / 2;
+    if (clusters < npairs) npairs = clusters;
+    if (prm.units_total < npairs) npairs = prm.units_total;
+    cfg.gridDim = dim3(2 * npairs);
+    // cooperative as well where the runtime accepts it together with clusters
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (!dev->no_coop_clusters) {
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tm_w2, tm_u, prm);
+        if (e == cudaSuccess) return DSPARK_OK;
+        if (e != cudaErrorInvalidValue && e != cudaErrorNotSupported &&
+            e != cudaErrorInvalidConfiguration)
+            return DSPARK_CUDA_ERROR;
+        cudaGetLastError();
+        dev->no_coop_clusters = true;
+    }
+    cfg.attrs = attr + 1;
     cfg.numAttrs = 1;
     return from_cuda(cudaLaunchKernelEx(&cfg, kern, tm_w2, tm_u, prm));
 }
@@ -291,6 +363,29 @@ int dspark_draft_step_rnn(const void *U, const int32_t *anchor, const void *W1, 
     if (!Whh) return DSPARK_INVALID_ARG;
     return launch_draft(U, anchor, W1, W2, Whh, B, gamma, V, r, mode, temperature, seed,
                         b_offset, x_out, logit_x_out, workspace, workspace_bytes, stream);
+}
+
+int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const void *W1,
+                                 const void *W2, const void *h, const void *w, float b_conf,
+                                 const float *T, int B, int gamma, int V, int r, int d, int mode,
+                                 float temperature, uint64_t seed, int b_offset, int32_t *x_out,
+                                 float *logit_x_out, float *c_out, float *P_out, void *workspace,
+                                 size_t workspace_bytes, dspark_stream_t stream)
+{
+    if (!h || !w || !T || !c_out || !P_out) return DSPARK_INVALID_ARG;
+    if (!aligned(h, 16) || !aligned(w, 16) || !aligned(T, 4) || !aligned(c_out, 4) ||
+        !aligned(P_out, 4))
+        return DSPARK_INVALID_ARG;
+    if (d < 8 || d % 8 != 0 || (d + r) * 2 > 200 * 1024 || gamma > dspark::conf::kMaxGamma)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    const ConfArgs conf{h, w, b_conf, T, d, c_out, P_out};
+    if (int st = launch_draft(U, anchor, W1, W2, nullptr, B, gamma, V, r, mode, temperature, seed,
+                              b_offset, x_out, logit_x_out, workspace, workspace_bytes, stream,
+                              &conf))
+        return st;
+    if (B <= 128) return DSPARK_OK;      // computed inside the draft launch
+    return dspark_confidence_sts(h, anchor, x_out, W1, w, b_conf, T, B, gamma, d, r, V, c_out,
+                                 P_out, stream);
 }
 
 int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x, const void *W1,

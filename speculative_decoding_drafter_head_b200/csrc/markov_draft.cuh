@@ -48,19 +48,21 @@ constexpr int kMaxUnits = 4;                      // 128 columns per MMA tile
 constexpr int kRank = 256;                        // r, the contraction length
 constexpr int kKSlice = 128;                      // W2 rows per ring stage
 constexpr int kKSlices = kRank / kKSlice;         // 2
-constexpr int kMaxW2Stages = 4;
+constexpr int kMaxW2Stages = 5;
 constexpr int kW2BoxBytes = 64 * kKSlice * 2;     // one TMA box: 64 columns x 128 rows (16 KB)
 constexpr int kW2StageBytes = 2 * kW2BoxBytes;    // 32 KB: 128 columns x 128 rows
-constexpr int kURingBytes = 64 * 1024;            // U boxes, rows x 64 columns each
 constexpr int kUMaxSlots = 16;
 constexpr int kAcc = 4;                           // TMEM accumulators of 128 columns
 constexpr int kAccCols = 128;
 constexpr uint32_t kTmemCols = 512;
-// A (M x 256 bf16) + W2 ring + U ring: M = 64 with 4 W2 stages or M = 128 with 3
-constexpr int kDynSmem = 224 * 1024 + 1024;       // + alignment slack
+// A (M x 256 bf16) + W2 ring + U ring in 224 KB (+ alignment slack)
+constexpr int kRingSmem = 224 * 1024;
+constexpr int kDynSmem = kRingSmem + 1024;
 constexpr int kEpiWarps = 8;                      // two per TMEM lane quadrant
 constexpr int kThreads = (kEpiWarps + 3) * 32;    // + W2 producer, U producer, MMA issuer
 constexpr int kWarpW2 = kEpiWarps, kWarpU = kEpiWarps + 1, kWarpMma = kEpiWarps + 2;
+constexpr int kWarpConf = kEpiWarps + 3;          // confidence head (fused instances only)
+constexpr int kThreadsConf = kThreads + 32;
 constexpr int kMaxB = 1024;
 constexpr int kMaxMTiles = kMaxB / 64;
 constexpr float kGumbelMax = 17.0f;               // above any noise value the epilogue makes
@@ -80,7 +82,7 @@ struct Params {
     unsigned int *abort_flag;    // set by any CTA that gives up, zeroed before launch
     int units_total;             // ceil(V / 32)
     int M;                       // requests per MMA tile: 64 (B <= 64) or 128
-    int w2_stages;               // W2 ring depth (4 when M = 64, else 3)
+    int w2_stages;               // W2 ring depth
     int ub;                      // rows of the U TMA box: min(B, M)
     int u_slots;                 // U ring depth (boxes of 64 columns)
     int u_slot_bytes;
@@ -90,6 +92,16 @@ struct Params {
     const uint16_t *Whh;         // [r][r] bf16
     float *state;                // [B][r] fp32, s_{k-1} then s_k (workspace)
     uint16_t *a_rows;            // [B][r] bf16 copy of s_k, the rows the gather reads
+    // confidence head fused in (kConf): z = w . [h_k ; W1[x_{k-1}]] + b_conf,
+    // c = sigmoid(z / T_k), P_k = P_{k-1} c
+    const uint16_t *h;           // [B][gamma][d] bf16
+    const uint16_t *wconf;       // [d + r] bf16
+    float b_conf;
+    const float *T;              // [gamma]
+    int d;
+    float *c_out, *P_out;        // [B][gamma]
+    float *zh;                   // [B][gamma] workspace: the hidden-state part of z
+    unsigned int *zh_done;       // workspace counter: CTAs whose zh share is written
 };
 
 struct Ctl {
@@ -102,6 +114,7 @@ struct Ctl {
     unsigned long long afull, aempty, drain;
     uint32_t tmem_base;
     int abort;
+    int go;          // verdict of the last grid barrier, shared by all epilogue threads
 };
 
 // A ring position: slot index and the parity of its current use.
@@ -465,10 +478,109 @@ __device__ __forceinline__ void box_update_m64(RowBest (&best)[2], const uint32_
     }
 }
 
+// 8 bf16 products of two 16-byte vectors added to acc (low half, then high half, of each
+// 32-bit word).
+__device__ __forceinline__ float dot8(const uint4 a, const uint4 b, float acc)
+{
+    acc = fmaf(bf16lo_to_f32(a.x), bf16lo_to_f32(b.x), acc);
+    acc = fmaf(bf16hi_to_f32(a.x), bf16hi_to_f32(b.x), acc);
+    acc = fmaf(bf16lo_to_f32(a.y), bf16lo_to_f32(b.y), acc);
+    acc = fmaf(bf16hi_to_f32(a.y), bf16hi_to_f32(b.y), acc);
+    acc = fmaf(bf16lo_to_f32(a.z), bf16lo_to_f32(b.z), acc);
+    acc = fmaf(bf16hi_to_f32(a.z), bf16hi_to_f32(b.z), acc);
+    acc = fmaf(bf16lo_to_f32(a.w), bf16lo_to_f32(b.w), acc);
+    acc = fmaf(bf16hi_to_f32(a.w), bf16hi_to_f32(b.w), acc);
+    return acc;
+}
+
+// Bounded wait of one thread until *ctr >= target (acquire); false on abort or time-out.
+__device__ __forceinline__ bool wait_counter(const unsigned int *ctr, uint32_t target,
+                                             const Params &p)
+{
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_u32(ctr) < target) {
+        if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) return false;
+        if (globaltimer_ns() - t0 > p.timeout_ns) {
+            record_error(DSPARK_TIMEOUT);
+            atomicExch(p.abort_flag, 1u);
+            return false;
+        }
+        __nanosleep(200);
+    }
+    return true;
+}
+
+// The confidence head, fused (gdymind.com "DSpark", section 5: a linear projection of the
+// backbone hidden state at position k and of the Markov embedding of the previous draft
+// token, a sigmoid, sequential temperature scaling, and the cumulative product of the
+// calibrated scores).  One warp of every CTA:
+//   1. z_h[b, k] = sum_i w[i] h[b, k-1, i] for the pairs n = b gamma + k - 1 with
+//      n = blockIdx.x (mod G), published with a release-add on a workspace counter;
+//   2. for k = 1..gamma, once the grid barrier of position k - 1 has passed (x_{k-1} is
+//      final): for the requests b = blockIdx.x (mod G), z = z_h + w[d..] . W1[x_{k-1}]
+//      + b_conf, c_k = 1 / (1 + exp(-z / T_k)), P_k = P_{k-1} c_k in fp32, k order.
+// It waits only on the grid barrier's counter, so it runs beside the drafting, off its
+// critical path.
+__device__ __forceinline__ void confidence_warp(const Params &p, int G)
+{
+    const int lane = threadIdx.x & 31;
+    const int n_pairs = p.B * p.gamma;
+    const int dv = p.d >> 3;                                    // 16-byte vectors of h
+    const uint4 *wv = reinterpret_cast<const uint4 *>(p.wconf);
+    for (int n = blockIdx.x; n < n_pairs; n += G) {
+        const uint4 *hk = reinterpret_cast<const uint4 *>(p.h + static_cast<size_t>(n) * p.d);
+        float a0 = 0.f, a1 = 0.f;
+        int i = lane;
+        for (; i + 32 < dv; i += 64) {                          // two vectors in flight per lane
+            const uint4 h0 = __ldcs(hk + i), h1 = __ldcs(hk + i + 32);
+            a0 = dot8(h0, __ldg(wv + i), a0);
+            a1 = dot8(h1, __ldg(wv + i + 32), a1);
+        }
+        if (i < dv) a0 = dot8(__ldcs(hk + i), __ldg(wv + i), a0);
+        const float z = warp_sum(a0 + a1);
+        if (lane == 0) p.zh[n] = z;
+    }
+    __syncwarp();
+    if (lane == 0) red_release_add_u32(p.zh_done, 1u);
+    bool ok = true;
+    if (lane == 0) ok = wait_counter(p.zh_done, static_cast<uint32_t>(G), p);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    const uint4 *wr = wv + dv;                                  // the W1-row part of w
+    const int rv = kRank >> 3;                                  // 32 vectors: one per lane
+    for (int k = 1; k <= p.gamma && ok; ++k) {
+        if (k >= 2 && lane == 0)                                // x_{k-1} final after barrier k-1
+            ok = wait_counter(p.barrier, static_cast<uint32_t>(k - 1) * static_cast<uint32_t>(G), p);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        const float Tk = __ldg(p.T + (k - 1));
+        for (int b = blockIdx.x; b < p.B; b += G) {
+            int tok = k == 1 ? __ldg(p.anchor + b)
+                             : static_cast<int>(argmax_key_index(
+                                   __ldcg(&p.slots[static_cast<size_t>(k - 2) * p.B + b])));
+            if (tok < 0 || tok >= p.V) {
+                if (lane == 0) record_error(DSPARK_INVALID_TOKEN);
+                tok = 0;
+            }
+            const uint4 *e = reinterpret_cast<const uint4 *>(p.W1 + static_cast<size_t>(tok) * kRank);
+            float zr = lane < rv ? dot8(__ldg(e + lane), __ldg(wr + lane), 0.f) : 0.f;
+            zr = warp_sum(zr);
+            if (lane == 0) {
+                const size_t o = static_cast<size_t>(b) * p.gamma + (k - 1);
+                const float z = __ldcg(p.zh + o) + zr + p.b_conf;
+                const float c = 1.0f / (1.0f + expf(-z / Tk));
+                const float P = k == 1 ? c : __fmul_rn(p.P_out[o - 1], c);
+                p.c_out[o] = c;
+                p.P_out[o] = P;
+            }
+        }
+    }
+}
+
 // kM is the MMA's M (64 when B <= 64, else 128); p.M equals it.  kRnn selects the RNN
-// head (p.Whh set); the Markov instances carry none of its code.
-template <int kM, bool kRnn>
-__global__ void __launch_bounds__(kThreads, 1)
+// head (p.Whh set); the Markov instances carry none of its code.  kConf adds the
+// confidence warp (Markov head only).
+template <int kM, bool kRnn, bool kConf = false>
+__global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
     markov_draft_kernel(const __grid_constant__ CUtensorMap tm_w2,
                         const __grid_constant__ CUtensorMap tm_u, const Params p)
 {
@@ -678,6 +790,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_drain(bar_drain, 0, p);
             }
         }
+    } else if (kConf && warp == kWarpConf) {
+        // ------------------------------------------------------------ confidence head
+        if constexpr (kConf) confidence_warp(p, G);
     } else {
         // ------------------------------------------------------------ epilogue (warps 0-7)
         const int q = warp & 3;                   // TMEM lane quadrant
@@ -689,8 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
         const int chunk = lane >> 3, unit = lane & 7;
         const int gather_rows = rq / 2;           // rows of the quadrant this warp gathers
-        Ring acc;
-        long long u_pos = 0;                      // U boxes consumed so far
+        Ring acc, ur;                             // accumulator and U box sequence
         uint32_t mt_count = 0;
         bool ok = true;
         int next_tok[kMaxMTiles];
@@ -733,28 +847,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // bounded grid barrier number nth (counted from 1 over the whole launch); false
         // once this CTA or any other gave up.  trace_k > 0 stamps the trace of position k.
+        // The verdict is taken by one thread and shared, so that every epilogue thread
+        // agrees on it; a warp that failed earlier marks the CTA as stopping first.
         auto grid_sync = [&](uint32_t nth, int trace_k) -> bool {
+            if (!ok) *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
             epi_sync();
-            if (threadIdx.x == 0 && ok && !*reinterpret_cast<volatile int *>(&ctl.abort)) {
-                red_release_add_u32(p.barrier, 1u);
-                if (trace_k > 0) DSPARK_TRACE_AT(trace_k, 4);
-                const uint32_t target =
-                    nth * static_cast<uint32_t>(G) + static_cast<uint32_t>(p.barrier_extra);
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_u32(p.barrier) < target) {
-                    if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
-                        *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
-                        break;
+            if (threadIdx.x == 0) {
+                bool good = !*reinterpret_cast<volatile int *>(&ctl.abort);
+                if (good) {
+                    red_release_add_u32(p.barrier, 1u);
+                    if (trace_k > 0) DSPARK_TRACE_AT(trace_k, 4);
+                    const uint32_t target =
+                        nth * static_cast<uint32_t>(G) + static_cast<uint32_t>(p.barrier_extra);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_u32(p.barrier) < target) {
+                        if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
+                            good = false;
+                            break;
+                        }
+                        if (globaltimer_ns() - t0 > p.timeout_ns) {
+                            give_up(ctl, p, DSPARK_TIMEOUT);
+                            good = false;
+                            break;
+                        }
                     }
-                    if (globaltimer_ns() - t0 > p.timeout_ns) {
-                        give_up(ctl, p, DSPARK_TIMEOUT);
-                        break;
-                    }
+                    if (trace_k > 0) DSPARK_TRACE_AT(trace_k, 5);
                 }
-                if (trace_k > 0) DSPARK_TRACE_AT(trace_k, 5);
+                if (!good) *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
+                ctl.go = good ? 1 : 0;
             }
             epi_sync();
-            return ok && !*reinterpret_cast<volatile int *>(&ctl.abort);
+            return *reinterpret_cast<volatile int *>(&ctl.go) != 0;
         };
         constexpr uint32_t bars_per_pos = kRnn ? 2u : 1u;
 
@@ -763,12 +886,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // holds columns 8l .. 8l + 7), the eight partial rows are summed through shared
         // memory, and thread t finishes element t.  The A tile's shared memory, free until
         // the gather that follows, holds s_{k-1} and the partial sums.
+        // After a failure it skips the work but keeps its named barriers.
         auto rnn_update = [&](int k) {
             float *scr = reinterpret_cast<float *>(dyn_smem + (sA - smem_u32(dyn_smem)));
             float *s_prev = scr;                          // [256]
             float *part = scr + kRank;                    // [8][256]
             const int t = threadIdx.x, w = t >> 5, ln = t & 31;
             for (int b = blockIdx.x; b < p.B; b += G) {
+                if (!ok) {
+                    epi_sync();
+                    epi_sync();
+                    epi_sync();
+                    continue;
+                }
                 int tok = k == 1 ? p.anchor[b]
                                  : static_cast<int>(argmax_key_index(
                                        __ldcg(&p.slots[static_cast<size_t>(k - 2) * p.B + b])));
@@ -809,22 +939,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             __threadfence();                  // the rows are read by every CTA after the barrier
         };
 
-        for (int k = 1; k <= p.gamma && ok; ++k) {
-            if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
+        // Every epilogue warp runs the same sequence of named barriers whatever happens:
+        // after a failed wait a warp only skips work, so that no bar.sync is left short.
+        for (int k = 1; k <= p.gamma; ++k) {
+            if (ok && !__all_sync(0xFFFFFFFFu, wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p)))
                 ok = false;
-                break;
-            }
             if constexpr (kRnn) {
                 rnn_update(k);
-                if (!grid_sync(static_cast<uint32_t>(2 * k - 1), 0)) {
-                    ok = false;
-                    break;
-                }
+                if (!grid_sync(static_cast<uint32_t>(2 * k - 1), 0)) ok = false;
             }
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 0);
-            gather(0);
+            if (ok) gather(0);
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 1);
-            for (int mt = 0; mt < num_mt && ok; ++mt) {
+            for (int mt = 0; mt < num_mt; ++mt) {
                 const int m0 = mt * M;
                 const int my_b = m0 + row;
                 // the next M tile's rows are gathered as soon as the MMA has released A, so
@@ -836,82 +963,84 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int b_glob = my_b + p.b_offset;
                 RowBest best;
                 RowBest best64[2];
-                for (int t = 0; t < ntiles && ok; ++t) {
+                for (int t = 0; t < ntiles; ++t) {
                     int first, count;
                     tile_span(t, n_units, ntiles, first, count);
+                    const int nbox = (count + 1) >> 1;
 #ifdef DSPARK_TRACE
                     const uint64_t tfw0 = globaltimer_ns();
 #endif
                     // warp-uniform outcome: tcgen05.ld below needs every lane of the warp
-                    if (!__all_sync(0xFFFFFFFFu,
-                                    wait_phase(bar_tfull + 8 * acc.slot, acc.phase, ctl, p))) {
+                    if (ok && !__all_sync(0xFFFFFFFFu,
+                                          wait_phase(bar_tfull + 8 * acc.slot, acc.phase, ctl, p)))
                         ok = false;
-                        break;
+                    if (ok) {
+                        tc_fence_after();
+                        if (threadIdx.x == 0 && mt == 0 && t == 0) DSPARK_TRACE_AT(k, 2);
+                        if (threadIdx.x == 0 && mt == num_mt - 1 && t == ntiles - 1) DSPARK_TRACE_AT(k, 21);
+                        if (threadIdx.x == 0 && t > 0) DSPARK_TRACE_ADD(k, 20, globaltimer_ns() - tfw0);
+#ifdef DSPARK_TRACE
+                        const uint64_t tbusy0 = globaltimer_ns();
+#endif
+                        // box i of the tile holds chunks 2i and 2i + 1; this warp takes boxes
+                        // i = half, half + 2, ... and reduces both chunks of a box together
+                        const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
+                        Ring my = ur;
+                        if (half) my.next(p.u_slots);
+                        for (int i = half; i < nbox; i += 2) {
+#ifdef DSPARK_TRACE
+                            const uint64_t tw2 = globaltimer_ns();
+#endif
+                            if (!__all_sync(0xFFFFFFFFu,
+                                            wait_phase(bar_u_full + 8 * my.slot, my.phase, ctl, p))) {
+                                ok = false;
+                                break;
+                            }
+                            if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 15, globaltimer_ns() - tw2);
+                            const uint32_t u_box = sU + my.slot * p.u_slot_bytes;
+                            if (active && M == 64) {
+                                uint32_t a[32];
+                                tmem_ld_16x256b_x8(t_acc + 2 * i * kUnit, a);
+                                tmem_wait_ld();
+                                box_update_m64(best64, a, 2 * i + 1 < count, u_box, ua64, ub64,
+                                               (u_begin + first + 2 * i) * kUnit, p, k,
+                                               r64 + p.b_offset, r64 + 8 + p.b_offset);
+                            } else if (active) {
+                                const bool two = 2 * i + 1 < count;
+                                uint32_t a0[32], a1[32];
+                                tmem_ld_32x32b_x32(t_acc + 2 * i * kUnit, a0);
+                                tmem_ld_32x32b_x32(t_acc + (two ? 2 * i + 1 : 2 * i) * kUnit, a1);
+                                tmem_wait_ld();
+                                box_update(best, a0, a1, two, u_box, urow,
+                                           (u_begin + first + 2 * i) * kUnit, p, k, b_glob);
+                            }
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar_u_empty + 8 * my.slot);
+                            my.next(p.u_slots);
+                            my.next(p.u_slots);
+                        }
+                        if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 19, globaltimer_ns() - tbusy0);
                     }
-                    tc_fence_after();
-                    if (threadIdx.x == 0 && mt == 0 && t == 0) DSPARK_TRACE_AT(k, 2);
-                    if (threadIdx.x == 0 && mt == num_mt - 1 && t == ntiles - 1) DSPARK_TRACE_AT(k, 21);
-                    if (threadIdx.x == 0 && t > 0) DSPARK_TRACE_ADD(k, 20, globaltimer_ns() - tfw0);
-#ifdef DSPARK_TRACE
-                    const uint64_t tbusy0 = globaltimer_ns();
-#endif
-                    // box i of the tile holds chunks 2i and 2i + 1; this warp takes boxes i = half,
-                    // half + 2, ... and reduces both chunks of a box together
-                    const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
-                    const int nbox = (count + 1) >> 1;
-                    for (int i = half; i < nbox; i += 2) {
-                        const long long pos = u_pos + i;
-                        const int slot = static_cast<int>(pos % p.u_slots);
-                        const uint32_t par = static_cast<uint32_t>((pos / p.u_slots) & 1);
-#ifdef DSPARK_TRACE
-                        const uint64_t tw2 = globaltimer_ns();
-#endif
-                        if (!__all_sync(0xFFFFFFFFu, wait_phase(bar_u_full + 8 * slot, par, ctl, p))) {
-                            ok = false;
-                            break;
-                        }
-                        if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 15, globaltimer_ns() - tw2);
-                        if (active && M == 64) {
-                            uint32_t a[32];
-                            tmem_ld_16x256b_x8(t_acc + 2 * i * kUnit, a);
-                            tmem_wait_ld();
-                            box_update_m64(best64, a, 2 * i + 1 < count, sU + slot * p.u_slot_bytes,
-                                           ua64, ub64, (u_begin + first + 2 * i) * kUnit, p, k,
-                                           r64 + p.b_offset, r64 + 8 + p.b_offset);
-                        } else if (active) {
-                            const bool two = 2 * i + 1 < count;
-                            uint32_t a0[32], a1[32];
-                            tmem_ld_32x32b_x32(t_acc + 2 * i * kUnit, a0);
-                            tmem_ld_32x32b_x32(t_acc + (two ? 2 * i + 1 : 2 * i) * kUnit, a1);
-                            tmem_wait_ld();
-                            box_update(best, a0, a1, two, sU + slot * p.u_slot_bytes, urow,
-                                       (u_begin + first + 2 * i) * kUnit, p, k, b_glob);
-                        }
+                    for (int i = 0; i < nbox; ++i) ur.next(p.u_slots);
+                    if (ok) {
+                        tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bar_u_empty + 8 * slot);
+                        if (lane == 0) mbar_arrive(bar_tempty + 8 * acc.slot);
                     }
-                    u_pos += nbox;
-                    if (threadIdx.x == 0) DSPARK_TRACE_ADD(k, 19, globaltimer_ns() - tbusy0);
-                    if (!ok) break;
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_tempty + 8 * acc.slot);
                     acc.next(kAcc);
-                    if (!next_gathered &&
+                    if (ok && !next_gathered &&
                         __all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty, (mt_count & 1u) ^ 1u))) {
                         gather(mt + 1);
                         next_gathered = true;
                     }
                 }
-                if (!ok) break;
-                if (!next_gathered) {
-                    if (!__all_sync(0xFFFFFFFFu,
-                                    wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p))) {
+                if (ok && !next_gathered) {
+                    if (__all_sync(0xFFFFFFFFu, wait_phase(bar_aempty, (mt_count & 1u) ^ 1u, ctl, p)))
+                        gather(mt + 1);
+                    else
                         ok = false;
-                        break;
-                    }
-                    gather(mt + 1);
                 }
+                if (!ok) continue;
                 if (M == 64) {
                     // the four threads of a row hold disjoint columns: combine, one atomic per row
 #pragma unroll
@@ -936,10 +1065,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // ---- grid barrier: every CTA has combined its rows of position k
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 3);
-            if (!grid_sync(static_cast<uint32_t>(k) * bars_per_pos, k)) {
-                ok = false;
-                break;
-            }
+            if (!grid_sync(static_cast<uint32_t>(k) * bars_per_pos, k)) ok = false;
+            if (!ok) continue;
             // ---- x_k of my rows: next gather's tokens; the owning CTA/half writes the outputs
             for (int mt = 0; mt < num_mt; ++mt) {
                 const int b = mt * M + row;

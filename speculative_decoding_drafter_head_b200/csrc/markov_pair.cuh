@@ -1,0 +1,647 @@
+// markov_pair.cuh -- the Markov head for large batches (B > 128) on CTA pairs.
+//
+// gdymind.com, "DSpark: DeepSeek's new speculative decoding work", section 4 ("Sequential
+// stage", "Markov head"): position k adds the transition bias W1[x_{k-1}] W2 (rank
+// r = 256) to the backbone's base logits U_k and picks x_k from them.  The arithmetic is
+// that of markov_draft_kernel; this kernel arranges it for many requests.
+//
+// With more than 128 requests the bias GEMM has several 128-row M tiles, and a single
+// CTA streams its whole W2 slice once per M tile.  Here the CTAs run as pairs (clusters
+// of two on one TPC) and every MMA is a pair MMA (tcgen05.mma.cta_group::2, M = 256): the
+// even CTA issues it, each CTA holds the A rows of its own 128 requests and half of the
+// W2 tile's columns, and each CTA's TMEM receives its 128 rows of the accumulator.  Every
+// W2 byte a CTA loads therefore serves 256 requests instead of 128.  Each pair owns a
+// contiguous vocabulary slice cut into 128-column tiles; for every position k and every
+// block of 256 requests it walks the tiles, alternating direction from one pass to the
+// next, so that the tiles read last are read again first and are still in L2.
+//
+// Per CTA: 16 epilogue warps (four per TMEM lane quadrant, one 32-column chunk of every
+// tile each), warp 16 the W2 producer (TMA, 64 columns x 128 K rows per stage), warp 17
+// the U producer (TMA, 128 rows x 64 columns per box), warp 18 the MMA issuer in the even
+// CTA and, in the odd CTA, the relay that tells the even CTA when the odd CTA's W2 stage
+// has landed.  Signals that cross the pair: the odd CTA's W2 arrivals (relayed), its A
+// gathers and its accumulator releases arrive on the even CTA's barriers; the even CTA's
+// MMA completions arrive on both CTAs' barriers through one pair commit.
+//
+// Selection as in markov_draft_kernel: greedy argmax with the smallest index on ties, or
+// Gumbel-max with Philox noise keyed (seed, request, position, vocabulary index).  Here the
+// Gumbel scores are taken in the log2 domain, l log2(e)/tau - log2(-log2 u), which is
+// log2(e) times the natural-log score minus a constant, so the chosen index is the same.
+// Rows are combined within the CTA through shared memory and across CTAs by a 64-bit
+// atomicMax; a bounded grid barrier ends each position.
+#pragma once
+#include "markov_draft.cuh"
+
+namespace dspark {
+namespace draft {
+namespace pairk {
+
+constexpr int kEpiWarps = 16;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kWarpW2 = kEpiWarps, kWarpU = kEpiWarps + 1, kWarpMma = kEpiWarps + 2;
+constexpr int kThreads = (kEpiWarps + 3) * 32;        // 608
+constexpr int kRows = 128;                            // requests per CTA per pass
+constexpr int kPairRows = 2 * kRows;                  // the pair MMA's M
+constexpr int kW2Stages = 5;
+constexpr int kW2StageBytes = 64 * kKSlice * 2;       // 64 columns x 128 K rows: 16 KB
+constexpr int kUSlots = 4;
+constexpr int kUSlotBytes = kRows * kUBoxCols * 2;    // 128 rows x 64 columns: 16 KB
+constexpr int kABytes = kRows * kRank * 2;            // 64 KB
+constexpr int kAChunkBytes = kRows * 128;             // 64 K-elements of A: 16 KB
+constexpr int kDynSmem = kABytes + kW2Stages * kW2StageBytes + kUSlots * kUSlotBytes + 1024;
+constexpr int kMaxPasses = kMaxB / kPairRows;         // 256-request blocks: 4
+constexpr int kChunks = 4;                            // 32-column chunks of a tile
+constexpr int kBoxWarps = 2 * 4;                      // warps reading one U box: 2 chunks x 4 quadrants
+constexpr float kLog2e = 1.4426950408889634f;
+// above any log2-domain noise value: -log2(-log2 u) <= -log2(2^-24 log2 e) < 23.5
+constexpr float kGumbel2Max = 24.0f;
+
+struct Ctl {
+    unsigned long long w2_full[kW2Stages];   // this CTA's W2 stage has landed (local TMA)
+    unsigned long long w2_peer[kW2Stages];   // even CTA: the odd CTA's stage has landed
+    unsigned long long w2_empty[kW2Stages];  // both: the pair MMAs have read the stage
+    unsigned long long u_full[kUSlots];
+    unsigned long long u_empty[kUSlots];
+    unsigned long long tfull[kAcc];          // both: the accumulator holds a tile
+    unsigned long long tempty[kAcc];         // even CTA: all 32 epilogue warps have read it
+    unsigned long long afull;                // even CTA: all 32 epilogue warps gathered A
+    unsigned long long aempty;               // both: the pair MMAs no longer read A
+    unsigned long long drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct Shared {
+    Ctl ctl;
+    unsigned long long part_key[kChunks][kRows];   // per chunk warp, before the CTA combine
+    float part_logit[kChunks][kRows];
+    unsigned long long cta_key[kMaxPasses][kRows];  // this CTA's best per row and pass
+    float cta_logit[kMaxPasses][kRows];
+    int tok[kMaxPasses][kRows];                     // x_{k-1} of this CTA's rows (-1: none)
+    int go;                                         // verdict of the last grid barrier
+};
+
+// Named barrier of the 16 epilogue warps.
+__device__ __forceinline__ void epi_sync512() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+__device__ __forceinline__ void give_up(Ctl &ctl, const Params &p, unsigned code)
+{
+    record_error(code);
+    *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
+    atomicExch(p.abort_flag, 1u);
+}
+
+// Bounded wait on an mbarrier phase; `cluster` selects acquire at cluster scope (for
+// barriers that the other CTA of the pair arrives on).  False once this CTA or any other
+// gave up, or the wait ran out.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl &ctl, const Params &p,
+                                         bool cluster = false)
+{
+    if (!cluster && mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (cluster ? mbar_try_wait_cluster(bar, parity, kWaitHintNs)
+                    : mbar_try_wait_sleep(bar, parity, kWaitHintNs))
+            return true;
+        if (*reinterpret_cast<volatile int *>(&ctl.abort) ||
+            *reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
+            *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > p.timeout_ns) {
+            give_up(ctl, p, DSPARK_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// The j-th tile of pass `pass`: forward on even passes, backward on odd ones.
+__device__ __forceinline__ int snake(int pass, int j, int ntiles)
+{
+    return (pass & 1) ? ntiles - 1 - j : j;
+}
+
+// ------------------------------------------------------------------ Philox, one request row
+// Philox4x32-10 (Salmon et al., SC'11) on the counter (x, y, z, 0), where y = k - 1 and
+// z = the request are fixed for a row: the parts of the first two rounds that depend only
+// on them are computed once per row and position.
+constexpr uint32_t kPhM0 = 0xD2511F53u, kPhM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhW0 = 0x9E3779B9u, kPhW1 = 0xBB67AE85u;
+
+struct RowNoise {
+    uint32_t r0, l1, h0p, l0p;
+};
+
+__device__ __forceinline__ RowNoise row_noise(uint32_t y, uint32_t z, uint32_t k0, uint32_t k1)
+{
+    RowNoise n;
+    n.r0 = __umulhi(kPhM1, z) ^ y ^ k0;     // word 0 after round 1
+    n.l1 = kPhM1 * z;                       // word 1 after round 1
+    n.h0p = __umulhi(kPhM0, n.r0);          // round 2 products of word 0
+    n.l0p = kPhM0 * n.r0;
+    (void)k1;
+    return n;
+}
+
+__device__ __forceinline__ uint4 philox_row(uint32_t x, const RowNoise &n, uint32_t k0,
+                                            uint32_t k1)
+{
+    const uint32_t hi0 = __umulhi(kPhM0, x), lo0 = kPhM0 * x;    // round 1
+    const uint32_t cz = hi0 ^ k1;
+    k0 += kPhW0;
+    k1 += kPhW1;
+    const uint32_t hi1 = __umulhi(kPhM1, cz), lo1 = kPhM1 * cz;   // round 2
+    uint4 c = make_uint4(hi1 ^ n.l1 ^ k0, lo1, n.h0p ^ lo0 ^ k1, n.l0p);
+#pragma unroll
+    for (int round = 2; round < 10; ++round) {
+        k0 += kPhW0;
+        k1 += kPhW1;
+        const uint32_t a0 = __umulhi(kPhM0, c.x), b0 = kPhM0 * c.x;
+        const uint32_t a1 = __umulhi(kPhM1, c.z), b1 = kPhM1 * c.z;
+        c = make_uint4(a1 ^ c.y ^ k0, b1, a0 ^ c.w ^ k1, b0);
+    }
+    return c;
+}
+
+// Log2-domain noise of one Philox word: u = ((w >> 9) + 0.5) 2^-23 (exact), and the result
+// is -log2(e2) with e2 = -log2 u, which equals log2(e) (-ln(-ln u)) - log2(log2 e).  e2 is
+// the hardware log2 except within 2^-6 of u = 1, where the hardware log2 loses relative
+// accuracy and e2 = log2(e) (t + t^2/2) with t = 1 - u (exact) is used instead: the
+// series -ln(1 - t) = t + t^2/2 + t^3/3 + ... cut after two terms, relative error < t^2/3.
+__device__ __forceinline__ float gumbel2_from_word(uint32_t w)
+{
+    const float u = fmaf(static_cast<float>(w >> 9), 0x1p-23f, 0x1p-24f);
+    const float t = 1.0f - u;
+    const float e_series = t * fmaf(t, 0.5f * kLog2e, kLog2e);
+    const float e_log = -__log2f(u);
+    const float e = (t < 0.015625f) ? e_series : e_log;
+    return -__log2f(e);
+}
+
+// One 32-column chunk of one request row: l = acc + U; greedy keeps the largest logit,
+// Gumbel-max the largest l c2 + noise (c2 = log2(e)/tau); strict improvement keeps the
+// smallest column on ties.
+__device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[32], uint32_t sU,
+                                             int row, int h, int v0, const Params &p,
+                                             const RowNoise &rn, float c2)
+{
+    float l[32];
+    add_u32(l, a, sU, row, h);
+    if (v0 + kUnit > p.V) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (v0 + i >= p.V) l[i] = -INFINITY;
+    }
+    if (p.mode == 0) {
+        const float mx = max32(l);
+        if (mx > best.s) {
+            best.v = static_cast<uint32_t>(v0 + first_index(l, mx));
+            best.s = mx;
+            best.l = mx;
+        }
+        return;
+    }
+    // exact pruning, one vote per warp: skip the noise when no row of the warp can beat its
+    // running best with the largest noise value
+    if (__all_sync(0xFFFFFFFFu, !(fmaf(max32(l), c2, kGumbel2Max) >= best.s))) return;
+    float s[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint4 w = philox_row(static_cast<uint32_t>((v0 >> 2) + q), rn, p.seed_lo, p.seed_hi);
+        s[4 * q + 0] = fmaf(l[4 * q + 0], c2, gumbel2_from_word(w.x));
+        s[4 * q + 1] = fmaf(l[4 * q + 1], c2, gumbel2_from_word(w.y));
+        s[4 * q + 2] = fmaf(l[4 * q + 2], c2, gumbel2_from_word(w.z));
+        s[4 * q + 3] = fmaf(l[4 * q + 3], c2, gumbel2_from_word(w.w));
+    }
+    const float mx = max32(s);
+    if (mx > best.s) {
+        const int idx = first_index(s, mx);
+        best.v = static_cast<uint32_t>(v0 + idx);
+        best.s = mx;
+        best.l = pick(l, idx);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    markov_pair_kernel(const __grid_constant__ CUtensorMap tm_w2,
+                       const __grid_constant__ CUtensorMap tm_u, const Params p)
+{
+    extern __shared__ uint8_t dyn_smem[];
+    __shared__ Shared sh;
+    Ctl &ctl = sh.ctl;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();          // 0: even CTA (issues the MMAs)
+    const bool lead = rank == 0;
+    const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+    const uint32_t sA = base;
+    const uint32_t sW2 = sA + kABytes;
+    const uint32_t sU = sW2 + kW2Stages * kW2StageBytes;
+
+    const int npairs = gridDim.x >> 1;
+    const int pair = blockIdx.x >> 1;
+    const int u_begin = static_cast<int>(static_cast<long long>(pair) * p.units_total / npairs);
+    const int u_end = static_cast<int>(static_cast<long long>(pair + 1) * p.units_total / npairs);
+    const int n_units = u_end - u_begin;
+    const int ntiles = (n_units + kMaxUnits - 1) / kMaxUnits;
+    const int npass = (p.B + kPairRows - 1) / kPairRows;   // 256-request blocks per position
+
+    const uint32_t bar_w2_full = smem_u32(&ctl.w2_full[0]);
+    const uint32_t bar_w2_peer = smem_u32(&ctl.w2_peer[0]);
+    const uint32_t bar_w2_empty = smem_u32(&ctl.w2_empty[0]);
+    const uint32_t bar_u_full = smem_u32(&ctl.u_full[0]);
+    const uint32_t bar_u_empty = smem_u32(&ctl.u_empty[0]);
+    const uint32_t bar_tfull = smem_u32(&ctl.tfull[0]);
+    const uint32_t bar_tempty = smem_u32(&ctl.tempty[0]);
+    const uint32_t bar_afull = smem_u32(&ctl.afull);
+    const uint32_t bar_aempty = smem_u32(&ctl.aempty);
+    const uint32_t bar_drain = smem_u32(&ctl.drain);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kW2Stages; ++s) {
+            mbar_init(bar_w2_full + 8 * s, 1);
+            mbar_init(bar_w2_peer + 8 * s, 1);
+            mbar_init(bar_w2_empty + 8 * s, 1);
+        }
+        for (int s = 0; s < kUSlots; ++s) {
+            mbar_init(bar_u_full + 8 * s, 1);
+            mbar_init(bar_u_empty + 8 * s, kBoxWarps);
+        }
+        for (int a = 0; a < kAcc; ++a) {
+            mbar_init(bar_tfull + 8 * a, 1);
+            mbar_init(bar_tempty + 8 * a, 2 * kEpiWarps);
+        }
+        mbar_init(bar_afull, 2 * kEpiWarps);
+        mbar_init(bar_aempty, 1);
+        mbar_init(bar_drain, 1);
+        ctl.abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc_pair(smem_u32(&ctl.tmem_base), kTmemCols);
+        tmem_relinquish_pair();
+    }
+    if (warp == kWarpW2 && lane == 0) {
+        tma_prefetch_desc(&tm_w2);
+        tma_prefetch_desc(&tm_u);
+    }
+    tc_fence_before();
+    cluster_sync();                  // both CTAs' barriers exist before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+
+    if (warp == kWarpW2) {
+        // ------------------------------------------------------------ W2 producer (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol_w2 = l2_policy_evict_last();
+            Ring w2;
+            long long issued = 0;
+            bool ok = true;
+            for (int k = 1; k <= p.gamma && ok; ++k)
+                for (int ps = 0; ps < npass && ok; ++ps) {
+                    const int pass = (k - 1) * npass + ps;
+                    for (int j = 0; j < ntiles && ok; ++j) {
+                        int first, count;
+                        tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                        // this CTA's half of the tile: columns rank * N/2 .. + N/2 (a 64-column box)
+                        const int x = (u_begin + first) * kUnit + static_cast<int>(rank) * count * (kUnit / 2);
+                        for (int ks = 0; ks < kKSlices; ++ks) {
+                            if (!wait_bar(bar_w2_empty + 8 * w2.slot, w2.phase ^ 1u, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t bar = bar_w2_full + 8 * w2.slot;
+                            mbar_arrive_expect_tx(bar, kW2StageBytes);
+                            tma_load_2d(sW2 + w2.slot * kW2StageBytes, &tm_w2, bar, x, ks * kKSlice,
+                                        pol_w2);
+                            ++issued;
+                            w2.next(kW2Stages);
+                        }
+                    }
+                }
+            // this CTA's copies land before exit; the last pair commits on w2_empty too
+            drain_ring(bar_w2_full, kW2Stages, issued, p);
+            drain_ring(bar_w2_empty, kW2Stages, issued, p);
+        }
+    } else if (warp == kWarpU) {
+        // ------------------------------------------------------------ U producer (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol_u = l2_policy_evict_first();
+            Ring ur;
+            long long issued = 0;
+            bool ok = true;
+            for (int k = 1; k <= p.gamma && ok; ++k)
+                for (int ps = 0; ps < npass && ok; ++ps) {
+                    const int pass = (k - 1) * npass + ps;
+                    const int row0 = ps * kPairRows + static_cast<int>(rank) * kRows;
+                    for (int j = 0; j < ntiles && ok; ++j) {
+                        int first, count;
+                        tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                        const int v0 = (u_begin + first) * kUnit;
+                        for (int u = 0; u < count; u += 2) {
+                            if (!wait_bar(bar_u_empty + 8 * ur.slot, ur.phase ^ 1u, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t bar = bar_u_full + 8 * ur.slot;
+                            mbar_arrive_expect_tx(bar, kUSlotBytes);
+                            tma_load_3d(sU + ur.slot * kUSlotBytes, &tm_u, bar, v0 + u * kUnit, k - 1,
+                                        row0, pol_u);
+                            ++issued;
+                            ur.next(kUSlots);
+                        }
+                    }
+                }
+            drain_ring(bar_u_full, kUSlots, issued, p);
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0 && !lead) {
+            // -------------------------------------------------------- relay (odd CTA)
+            // tell the even CTA when each of this CTA's W2 stages has landed
+            const uint32_t peer_bar0 = mapa_shared(bar_w2_peer, 0);
+            Ring w2;
+            bool ok = true;
+            for (int k = 1; k <= p.gamma && ok; ++k)
+                for (int ps = 0; ps < npass && ok; ++ps)
+                    for (int j = 0; j < ntiles * kKSlices && ok; ++j) {
+                        if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_cluster(peer_bar0 + 8 * w2.slot);
+                        w2.next(kW2Stages);
+                    }
+        } else if (lane == 0) {
+            // -------------------------------------------------------- pair MMA issuer (even CTA)
+            Ring w2, acc;
+            const uint64_t a_desc0 = smem_desc(sA, 1024, 1024, kSwizzle128B);
+            const uint64_t b_desc0 = smem_desc(sW2, kW2StageBytes, 1024, kSwizzle128B);
+            const uint16_t both = 0x3;
+            uint32_t a_count = 0;
+            bool issued_any = false;
+            bool ok = true;
+            for (int k = 1; k <= p.gamma && ok; ++k)
+                for (int ps = 0; ps < npass && ok; ++ps) {
+                    const int pass = (k - 1) * npass + ps;
+                    if (!wait_bar(bar_afull, a_count & 1u, ctl, p, true)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int j = 0; j < ntiles && ok; ++j) {
+                        int first, count;
+                        tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                        const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(kPairRows),
+                                                              static_cast<uint32_t>(count * kUnit), 1);
+                        if (!wait_bar(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p, true)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
+                        for (int ks = 0; ks < kKSlices; ++ks) {
+                            if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p) ||
+                                !wait_bar(bar_w2_peer + 8 * w2.slot, w2.phase, ctl, p, true)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint64_t a_k = a_desc0 + static_cast<uint64_t>((2 * ks * kAChunkBytes) >> 4);
+                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((w2.slot * kW2StageBytes) >> 4);
+#pragma unroll
+                            for (int kk = 0; kk < kKSlice / 16; ++kk) {
+                                const uint64_t a_desc =
+                                    a_k + static_cast<uint64_t>(((kk >> 2) * kAChunkBytes + (kk & 3) * 32) >> 4);
+                                const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
+                                umma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (ks | kk) ? 1u : 0u);
+                            }
+                            issued_any = true;
+                            umma_commit_pair_mask(bar_w2_empty + 8 * w2.slot, both);
+                            w2.next(kW2Stages);
+                        }
+                        if (!ok) break;
+                        umma_commit_pair_mask(bar_tfull + 8 * acc.slot, both);
+                        acc.next(kAcc);
+                    }
+                    if (!ok) break;
+                    umma_commit_pair_mask(bar_aempty, both);
+                    ++a_count;
+                }
+            if (issued_any) {
+                umma_commit_pair(bar_drain);
+                wait_drain(bar_drain, 0, p);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 0-15)
+        // Every epilogue warp runs the same sequence of named barriers whatever happens:
+        // after a failed wait a warp only skips work (waits, loads, copies), so that no
+        // bar.sync is ever left short of arrivals.
+        const int et = threadIdx.x;                       // 0 .. 511
+        const int q = warp & 3;                           // TMEM lane quadrant
+        const int c = warp >> 2;                          // chunk of every tile: columns 32c ..
+        const int row = q * 32 + lane;                    // row of this CTA's 128
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t afull_lead = mapa_shared(bar_afull, 0);
+        const uint32_t tempty_lead = mapa_shared(bar_tempty, 0);
+        const float c2 = p.inv_tau * kLog2e;
+        Ring acc, ur;
+        uint32_t a_count = 0;
+        bool ok = true;                                   // uniform within a warp
+
+        for (int i = et; i < kMaxPasses * kRows; i += kEpiThreads) {
+            const int ps = i / kRows, r = i % kRows;
+            const int b = ps * kPairRows + static_cast<int>(rank) * kRows + r;
+            sh.tok[ps][r] = (ps < npass && b < p.B) ? checked_token(p.anchor[b], p.V) : -1;
+        }
+        epi_sync512();
+
+        // this warp's share of the A gather of pass ps: rows 8 warp .. + 7, lane l copies 8
+        // of the 32 16-byte pieces of row 8 warp + l/4 (zeros for rows without a request)
+        auto gather = [&](int ps) {
+            const int r = 8 * warp + (lane >> 2);
+            const int tok = sh.tok[ps][r];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int unit = (lane & 3) * 8 + i;                 // 16-byte piece of the row
+                const uint32_t dst = sA + (unit >> 3) * kAChunkBytes + r * 128 +
+                                     (((unit & 7) ^ (r & 7)) << 4);
+                if (tok >= 0)
+                    cp_async_16(dst, p.W1 + static_cast<size_t>(tok) * kRank + unit * 8);
+                else
+                    sts128_zero(dst);
+            }
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (lead) mbar_arrive(bar_afull);
+                else mbar_arrive_cluster(afull_lead);
+            }
+            ++a_count;
+        };
+
+        // bounded grid barrier number nth; the verdict is taken by one thread and shared, so
+        // that all epilogue threads agree on it
+        auto grid_sync = [&](uint32_t nth) -> bool {
+            if (!ok) *reinterpret_cast<volatile int *>(&ctl.abort) = 1;   // this warp failed: stop
+            epi_sync512();
+            if (et == 0) {
+                bool good = !*reinterpret_cast<volatile int *>(&ctl.abort);
+                if (good) {
+                    red_release_add_u32(p.barrier, 1u);
+                    const uint32_t target = nth * static_cast<uint32_t>(gridDim.x) +
+                                            static_cast<uint32_t>(p.barrier_extra);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_u32(p.barrier) < target) {
+                        if (*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
+                            good = false;
+                            break;
+                        }
+                        if (globaltimer_ns() - t0 > p.timeout_ns) {
+                            give_up(ctl, p, DSPARK_TIMEOUT);
+                            good = false;
+                            break;
+                        }
+                    }
+                }
+                if (!good) *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
+                sh.go = good ? 1 : 0;
+            }
+            epi_sync512();
+            return sh.go != 0;
+        };
+
+        for (int k = 1; k <= p.gamma; ++k) {
+            if (ok) {
+                // L2 prefetch of the W1 rows of the later passes of this position (4 lines a row)
+                const int r = 8 * warp + (lane >> 2);
+                for (int ps = 1; ps < npass; ++ps) {
+                    const int tok = sh.tok[ps][r];
+                    if (tok >= 0) prefetch_l2(p.W1 + static_cast<size_t>(tok) * kRank + (lane & 3) * 64);
+                }
+                if (__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty, (a_count & 1u) ^ 1u, ctl, p)))
+                    gather(0);
+                else
+                    ok = false;
+            }
+            for (int ps = 0; ps < npass; ++ps) {
+                const int pass = (k - 1) * npass + ps;
+                const int b_row = ps * kPairRows + static_cast<int>(rank) * kRows + row;
+                const bool active = ps * kPairRows + static_cast<int>(rank) * kRows + q * 32 < p.B;
+                const RowNoise rn = row_noise(static_cast<uint32_t>(k - 1),
+                                              static_cast<uint32_t>(b_row + p.b_offset), p.seed_lo,
+                                              p.seed_hi);
+                bool next_gathered = ps + 1 >= npass;
+                RowBest best;
+                for (int j = 0; j < ntiles; ++j) {
+                    int first, count;
+                    tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                    const int nbox = (count + 1) >> 1;
+                    const int box = c >> 1;
+                    // warp-uniform: tcgen05.ld below needs every lane of the warp
+                    if (ok && !__all_sync(0xFFFFFFFFu,
+                                          wait_bar(bar_tfull + 8 * acc.slot, acc.phase, ctl, p)))
+                        ok = false;
+                    if (ok && box < nbox) {
+                        tc_fence_after();
+                        Ring my = ur;
+                        for (int i = 0; i < box; ++i) my.next(kUSlots);
+                        if (__all_sync(0xFFFFFFFFu, wait_bar(bar_u_full + 8 * my.slot, my.phase, ctl, p))) {
+                            if (active && c < count) {
+                                uint32_t a[32];
+                                tmem_ld_32x32b_x32(
+                                    t_lane + static_cast<uint32_t>(acc.slot * kAccCols + c * kUnit), a);
+                                tmem_wait_ld();
+                                chunk_update(best, a, sU + my.slot * kUSlotBytes, row, c & 1,
+                                             (u_begin + first + c) * kUnit, p, rn, c2);
+                            }
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar_u_empty + 8 * my.slot);
+                        } else {
+                            ok = false;
+                        }
+                    }
+                    for (int i = 0; i < nbox; ++i) ur.next(kUSlots);
+                    if (ok) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (lead) mbar_arrive(bar_tempty + 8 * acc.slot);
+                            else mbar_arrive_cluster(tempty_lead + 8 * acc.slot);
+                        }
+                    }
+                    acc.next(kAcc);
+                    // the next pass's rows are gathered as soon as the MMAs have released A
+                    if (ok && !next_gathered &&
+                        __all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty, (a_count & 1u) ^ 1u))) {
+                        gather(ps + 1);
+                        next_gathered = true;
+                    }
+                }
+                if (ok && !next_gathered) {
+                    if (__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty, (a_count & 1u) ^ 1u, ctl, p)))
+                        gather(ps + 1);
+                    else
+                        ok = false;
+                }
+                // combine the four chunk warps of each row, one atomic per row and CTA
+                sh.part_key[c][row] = argmax_key(best.s, best.v);
+                sh.part_logit[c][row] = best.l;
+                epi_sync512();
+                if (c == 0) {
+                    unsigned long long kb = sh.part_key[0][row];
+                    float lb = sh.part_logit[0][row];
+#pragma unroll
+                    for (int i = 1; i < kChunks; ++i) {
+                        const unsigned long long ki = sh.part_key[i][row];
+                        if (ki > kb) {
+                            kb = ki;
+                            lb = sh.part_logit[i][row];
+                        }
+                    }
+                    sh.cta_key[ps][row] = kb;
+                    sh.cta_logit[ps][row] = lb;
+                    if (ok && b_row < p.B)
+                        atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + b_row], kb);
+                }
+                epi_sync512();
+            }
+
+            // ---- grid barrier: every CTA has combined its rows of position k
+            if (!grid_sync(static_cast<uint32_t>(k))) ok = false;
+            // ---- x_k of this CTA's rows: the next gather's tokens; the owner writes the outputs
+            if (ok) {
+                for (int i = et; i < npass * kRows; i += kEpiThreads) {
+                    const int ps = i / kRows, r = i % kRows;
+                    const int b = ps * kPairRows + static_cast<int>(rank) * kRows + r;
+                    if (b >= p.B) continue;
+                    const size_t o = static_cast<size_t>(k - 1) * p.B + b;
+                    const unsigned long long key = __ldcg(&p.slots[o]);
+                    const int tok = static_cast<int>(argmax_key_index(key));
+                    sh.tok[ps][r] = checked_token(tok, p.V);
+                    if (key == sh.cta_key[ps][r]) {
+                        p.x_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = tok;
+                        p.logit_out[static_cast<size_t>(b) * p.gamma + (k - 1)] = sh.cta_logit[ps][r];
+                    }
+                }
+            }
+            epi_sync512();
+        }
+        // the last pair commit on aempty may still be arriving on this CTA's barrier
+        if (ok) wait_drain(bar_aempty, (a_count & 1u) ^ 1u, p);
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync();                  // no cross-CTA signal is in flight past this point
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace pairk
+}  // namespace draft
+}  // namespace dspark

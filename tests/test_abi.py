@@ -67,6 +67,27 @@ def test_draft_step_host_checks():
     assert call(wsb=100) == 3
 
 
+def test_draft_confidence_step_host_checks():
+    lib = ds.load()
+    f = lib.dspark_draft_confidence_step
+    args = dict(U=_FAKE, anchor=_FAKE, W1=_FAKE, W2=_FAKE, h=_FAKE, w=_FAKE, b_conf=1.0, T=_FAKE,
+                B=64, gamma=16, V=151936, r=256, d=4096, mode=0, temperature=1.0, seed=0,
+                b_offset=0, x=_FAKE, lx=_FAKE, c=_FAKE, P=_FAKE, ws=_FAKE, wsb=1 << 30, stream=None)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return f(a["U"], a["anchor"], a["W1"], a["W2"], a["h"], a["w"], a["b_conf"], a["T"], a["B"],
+                 a["gamma"], a["V"], a["r"], a["d"], a["mode"], a["temperature"], a["seed"],
+                 a["b_offset"], a["x"], a["lx"], a["c"], a["P"], a["ws"], a["wsb"], a["stream"])
+
+    assert call(h=None) == 1 and call(P=None) == 1
+    assert call(h=C.c_void_p(0x10008)) == 1          # not 16-byte aligned
+    assert call(d=1020) == 2
+    assert call(U=None) == 1                          # the drafting checks apply as well
+    assert call(B=1025) == 2
+    assert call(wsb=100) == 3
+
+
 def test_schedule_and_verify_host_checks():
     lib = ds.load()
     s = lib.dspark_schedule_prefix
