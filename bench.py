@@ -40,7 +40,8 @@ import synth  # noqa: E402
 PARITY_MACS = 3.5e11          # oracle multiply-adds spent on the bench line's parity check
 METRIC = "draft tokens/s (Markov head+confidence+schedule+verify); % of HBM/TC roofline"
 UNIT = "tokens/s"
-DRAFT_SRC = os.path.join(ROOT, "speculative_decoding_drafter_head_b200", "csrc", "markov_draft.cuh")
+DRAFT_SRCS = [os.path.join(ROOT, "speculative_decoding_drafter_head_b200", "csrc", f)
+              for f in ("markov_draft.cuh", "markov_pair.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "markov_draft_traffic.json")
 
 
@@ -57,8 +58,10 @@ def _kernel_sha():
     """Hash of the draft kernel's source with comments and blank space removed, so that the
     committed DRAM-traffic figure stays attached to the code it was measured on."""
     import re
-    with open(DRAFT_SRC, encoding="utf-8") as f:
-        src = f.read()
+    src = ""
+    for path in DRAFT_SRCS:
+        with open(path, encoding="utf-8") as f:
+            src += f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
     src = re.sub(r"\s+", " ", src).strip()
@@ -447,29 +450,43 @@ def main():
         lsched = pipeline.LaggedScheduler(B * world, gamma, Tstep, lag=2)
     step_no = [0]
 
+    # the Markov head drafts and scores in one call (one launch for B <= 128); the RNN
+    # head drafts, then the confidence kernel scores
+    fused = not rnn
+
+    def draft_and_score(P_dst):
+        if fused:
+            ds.draft_confidence_step(U, anchor, W1, W2, h, w, wl.b_conf, T, x, lx, c, P_dst, ws,
+                                     mode=wl.mode, temperature=wl.tau, seed=wl.seed, b_offset=b0)
+        else:
+            draft(mode=wl.mode, temperature=wl.tau, seed=wl.seed, b_offset=b0)
+
+    def score(P_dst):
+        if not fused:
+            ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P_dst)
+
     def step(record=None):
         t = step_no[0]
         step_no[0] += 1
         e0 = e1 = None
+        P_dst = lsched.scores(t) if lagged and world == 1 else P
         if record is not None:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        draft(mode=wl.mode, temperature=wl.tau, seed=wl.seed, b_offset=b0)
+        draft_and_score(P_dst)
         if record is not None:
             e1.record(stream)
             record.append((e0, e1))
         if lagged:
             lsched.begin_step(t)                   # overlaps the confidence kernel
+            score(P_dst)
             if world > 1:
-                ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P)
                 sharding.gather_scores(P, out=lsched.scores(t))
-            else:
-                ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, lsched.scores(t))
             Lt = lsched.lengths(t, workspace=ws)
             Lloc = sharding.local_lengths(Lt, rank, B) if world > 1 else Lt
         else:
-            ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P)
+            score(P)
             if world > 1:
                 sharding.gather_scores(P, out=Pg)
                 ds.schedule_prefix(Pg, Tstep, Lg, Nst, obj, ws)
@@ -545,11 +562,30 @@ def main():
                 "P": P.cpu().numpy(), "L": last_L[0].cpu().numpy(), "N": int(Nst.item()),
                 "F": float(obj.item()), "acc": acc.cpu().numpy(), "bonus": bonus.cpu().numpy()}
 
-    # the draft kernel alone, for its roofline (same inputs, L2 flushed before each launch)
+    # the draft call alone, for its roofline (same inputs, L2 flushed before each launch),
+    # replayed as a CUDA graph so that no host time falls between the events
+    g_draft = None
+    if not args.eager:
+        try:
+            g_draft = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_draft):
+                draft_and_score(P)
+        except Exception:                                  # noqa: BLE001
+            torch.cuda.synchronize()
+            g_draft = None
     for _ in range(args.steps):
         flush.zero_()
-        step(ev_draft)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        if g_draft is not None:
+            g_draft.replay()
+        else:
+            draft_and_score(P)
+        e1.record(stream)
+        ev_draft.append((e0, e1))
     torch.cuda.synchronize()
+    g_draft = None
     draft_ms = [a.elapsed_time(b) for a, b in ev_draft]
 
     # ---------------- end to end through the public API with host buffers
@@ -607,7 +643,8 @@ def main():
 
     if rank == 0:
         hbm_gbs, tflops, peak_kind = _peaks()
-        algo_bytes = gamma * (wl.r * V * 2 + B * V * 2)          # W2 + U_k per position
+        # W2 + U_k per position; with the confidence head in the same timed call, h as well
+        algo_bytes = gamma * (wl.r * V * 2 + B * V * 2) + (B * gamma * wl.d * 2 if fused else 0)
         achieved = algo_bytes / (draft_mean / 1e3) / 1e9
         flops = gamma * 2.0 * B * wl.r * V
         t_hbm = algo_bytes / (hbm_gbs * 1e9)
@@ -615,7 +652,8 @@ def main():
         roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "achieved": achieved,
                 "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                 "traffic": None if rnn else _traffic_per_launch(wl.name),
-                "kernel": "markov_draft_kernel",
+                "kernel": ("markov_pair_kernel" if B > 128 and not rnn else "markov_draft_kernel")
+                + (" + confidence head" if fused else ""),
                 "kernel_ms": draft_mean, "algorithmic_bytes": algo_bytes,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s"}
@@ -641,7 +679,7 @@ def main():
             "parity": parity,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (3 if fused and B <= 128 else 4) * args.steps,
             "cuda_graph": graph is not None,
             "schedule": "lagged by 2 steps, side stream" if lagged else "this step's scores",
             "head": args.head,

@@ -47,10 +47,42 @@ struct DeviceInfo {
     int sms = 0;
     int major = 0;
     bool no_coop_clusters = false;   // the runtime refused a cooperative cluster launch
+    // draft-kernel attributes and the pair kernel's resident clusters, valid for the CUDA
+    // context with this id (0: none yet); a new context (after a device reset) re-sets them
+    unsigned long long draft_ctx = 0;
+    int pair_clusters = 0;
 };
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current CUDA context (0 if unavailable).
+unsigned long long current_ctx_id()
+{
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
 constexpr int kMaxDevices = 64;
-constexpr int kW2StagesM64 = 5;   // W2 ring depth of the M = 64 instance (32 KB stages)
+constexpr int kW2StagesM64 = 4;   // W2 ring depth of the M = 64 instance (32 KB stages)
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -239,9 +271,28 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
                            : D::markov_draft_kernel<128, false, true>)
                 : (M == 64 ? D::markov_draft_kernel<64, false> : D::markov_draft_kernel<128, false>);
     const int dyn_smem = pair ? D::pairk::kDynSmem : D::kDynSmem;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem) !=
-        cudaSuccess)
-        return DSPARK_CUDA_ERROR;
+    {
+        // every instance's shared-memory limit, once per CUDA context (a device reset makes
+        // a new context, with a new id, and the attributes are set again)
+        const unsigned long long ctx = current_ctx_id();
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        if (ctx == 0 || dev->draft_ctx != ctx) {
+            void (*const all[])(const CUtensorMap, const CUtensorMap, const D::Params) = {
+                D::markov_draft_kernel<64, false>, D::markov_draft_kernel<128, false>,
+                D::markov_draft_kernel<64, true>, D::markov_draft_kernel<128, true>,
+                D::markov_draft_kernel<64, false, true>, D::markov_draft_kernel<128, false, true>};
+            for (auto f : all)
+                if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         D::kDynSmem) != cudaSuccess)
+                    return DSPARK_CUDA_ERROR;
+            if (cudaFuncSetAttribute(D::pairk::markov_pair_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     D::pairk::kDynSmem) != cudaSuccess)
+                return DSPARK_CUDA_ERROR;
+            dev->pair_clusters = 0;
+            dev->draft_ctx = ctx;
+        }
+    }
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     D::Params prm;
@@ -315,10 +366,13 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     cfg.gridDim = dim3(dev->sms & ~1);
     cfg.attrs = attr + 1;
     cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
-        cudaGetLastError();
-        return DSPARK_CUDA_ERROR;
+    int clusters = dev->pair_clusters;
+    if (clusters < 1) {
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+            cudaGetLastError();
+            return DSPARK_CUDA_ERROR;
+        }
+        dev->pair_clusters = clusters;
     }
     int npairs = dev->sms / 2;
     if (clusters < npairs) npairs = clusters;

@@ -10,7 +10,10 @@
 // of two on one TPC) and every MMA is a pair MMA (tcgen05.mma.cta_group::2, M = 256): the
 // even CTA issues it, each CTA holds the A rows of its own 128 requests and half of the
 // W2 tile's columns, and each CTA's TMEM receives its 128 rows of the accumulator.  Every
-// W2 byte a CTA loads therefore serves 256 requests instead of 128.  Each pair owns a
+// W2 byte a CTA loads therefore serves 256 requests instead of 128.  The A rows sit in
+// tensor memory (written there by the epilogue warps with tcgen05.st), so the tensor core
+// reads only W2 from shared memory, whose bandwidth the TMA copies and the epilogue's U
+// reads share.  Each pair owns a
 // contiguous vocabulary slice cut into 128-column tiles; for every position k and every
 // block of 256 requests it walks the tiles, alternating direction from one pass to the
 // next, so that the tiles read last are read again first and are still in L2.
@@ -42,13 +45,15 @@ constexpr int kWarpW2 = kEpiWarps, kWarpU = kEpiWarps + 1, kWarpMma = kEpiWarps 
 constexpr int kThreads = (kEpiWarps + 3) * 32;        // 608
 constexpr int kRows = 128;                            // requests per CTA per pass
 constexpr int kPairRows = 2 * kRows;                  // the pair MMA's M
-constexpr int kW2Stages = 5;
+constexpr int kW2Stages = 7;
 constexpr int kW2StageBytes = 64 * kKSlice * 2;       // 64 columns x 128 K rows: 16 KB
-constexpr int kUSlots = 4;
+constexpr int kUSlots = 6;
 constexpr int kUSlotBytes = kRows * kUBoxCols * 2;    // 128 rows x 64 columns: 16 KB
-constexpr int kABytes = kRows * kRank * 2;            // 64 KB
-constexpr int kAChunkBytes = kRows * 128;             // 64 K-elements of A: 16 KB
-constexpr int kDynSmem = kABytes + kW2Stages * kW2StageBytes + kUSlots * kUSlotBytes + 1024;
+constexpr int kDynSmem = kW2Stages * kW2StageBytes + kUSlots * kUSlotBytes + 1024;
+// TMEM (512 columns): three 128-column accumulators, then A = W1[x_{k-1}] of the CTA's
+// 128 rows (row m in lane m, K = 256 bf16 packed two per column: 128 columns)
+constexpr int kPairAcc = 3;
+constexpr uint32_t kACol = kPairAcc * kAccCols;       // 384
 constexpr int kMaxPasses = kMaxB / kPairRows;         // 256-request blocks: 4
 constexpr int kChunks = 4;                            // 32-column chunks of a tile
 constexpr int kBoxWarps = 2 * 4;                      // warps reading one U box: 2 chunks x 4 quadrants
@@ -62,8 +67,8 @@ struct Ctl {
     unsigned long long w2_empty[kW2Stages];  // both: the pair MMAs have read the stage
     unsigned long long u_full[kUSlots];
     unsigned long long u_empty[kUSlots];
-    unsigned long long tfull[kAcc];          // both: the accumulator holds a tile
-    unsigned long long tempty[kAcc];         // even CTA: all 32 epilogue warps have read it
+    unsigned long long tfull[kPairAcc];      // both: the accumulator holds a tile
+    unsigned long long tempty[kPairAcc];     // even CTA: all 32 epilogue warps have read it
     unsigned long long afull;                // even CTA: all 32 epilogue warps gathered A
     unsigned long long aempty;               // both: the pair MMAs no longer read A
     unsigned long long drain;
@@ -81,6 +86,20 @@ struct Shared {
     int go;                                         // verdict of the last grid barrier
 };
 
+// Optional per-tile timeline (build with -DDSPARK_TRACE): for position 2, pass 0, tile j
+// and event e, a %globaltimer stamp in g_trace[(blockIdx.x * 64 + j) * 32 + e].
+#ifdef DSPARK_TRACE
+#define PAIR_TRACE(k, ps, j, e)                                                               \
+    do {                                                                                      \
+        if ((k) == 2 && (ps) == 0 && (j) < 64 && blockIdx.x < 256)                            \
+            g_trace[(blockIdx.x * 64 + (j)) * 32 + (e)] = globaltimer_ns();                   \
+    } while (0)
+#else
+#define PAIR_TRACE(k, ps, j, e) \
+    do {                        \
+    } while (0)
+#endif
+
 // Named barrier of the 16 epilogue warps.
 __device__ __forceinline__ void epi_sync512() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
@@ -97,7 +116,7 @@ __device__ __forceinline__ void give_up(Ctl &ctl, const Params &p, unsigned code
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl &ctl, const Params &p,
                                          bool cluster = false)
 {
-    if (!cluster && mbar_try_wait(bar, parity)) return true;
+    if (cluster ? mbar_try_wait_cluster(bar, parity, 0) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (cluster ? mbar_try_wait_cluster(bar, parity, kWaitHintNs)
@@ -235,8 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t rank = cluster_ctarank();          // 0: even CTA (issues the MMAs)
     const bool lead = rank == 0;
     const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
-    const uint32_t sA = base;
-    const uint32_t sW2 = sA + kABytes;
+    const uint32_t sW2 = base;
     const uint32_t sU = sW2 + kW2Stages * kW2StageBytes;
 
     const int npairs = gridDim.x >> 1;
@@ -268,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_u_full + 8 * s, 1);
             mbar_init(bar_u_empty + 8 * s, kBoxWarps);
         }
-        for (int a = 0; a < kAcc; ++a) {
+        for (int a = 0; a < kPairAcc; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
             mbar_init(bar_tempty + 8 * a, 2 * kEpiWarps);
         }
@@ -311,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ok = false;
                                 break;
                             }
+                            PAIR_TRACE(k, ps, j, 8 + ks);
                             const uint32_t bar = bar_w2_full + 8 * w2.slot;
                             mbar_arrive_expect_tx(bar, kW2StageBytes);
                             tma_load_2d(sW2 + w2.slot * kW2StageBytes, &tm_w2, bar, x, ks * kKSlice,
@@ -344,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ok = false;
                                 break;
                             }
+                            PAIR_TRACE(k, ps, j, 10 + u / 2);
                             const uint32_t bar = bar_u_full + 8 * ur.slot;
                             mbar_arrive_expect_tx(bar, kUSlotBytes);
                             tma_load_3d(sU + ur.slot * kUSlotBytes, &tm_u, bar, v0 + u * kUnit, k - 1,
@@ -369,13 +389,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        mbar_arrive_cluster(peer_bar0 + 8 * w2.slot);
+                        PAIR_TRACE(k, ps, j / kKSlices, 12 + (j & 1));
+                        mbar_arrive_remote(peer_bar0 + 8 * w2.slot);
                         w2.next(kW2Stages);
                     }
         } else if (lane == 0) {
             // -------------------------------------------------------- pair MMA issuer (even CTA)
             Ring w2, acc;
-            const uint64_t a_desc0 = smem_desc(sA, 1024, 1024, kSwizzle128B);
             const uint64_t b_desc0 = smem_desc(sW2, kW2StageBytes, 1024, kSwizzle128B);
             const uint16_t both = 0x3;
             uint32_t a_count = 0;
@@ -394,10 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
                         const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(kPairRows),
                                                               static_cast<uint32_t>(count * kUnit), 1);
+                        PAIR_TRACE(k, ps, j, 0);
                         if (!wait_bar(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p, true)) {
                             ok = false;
                             break;
                         }
+                        PAIR_TRACE(k, ps, j, 1);
                         tc_fence_after();
                         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
                         for (int ks = 0; ks < kKSlices; ++ks) {
@@ -406,15 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ok = false;
                                 break;
                             }
+                            PAIR_TRACE(k, ps, j, 2 + ks);
                             tc_fence_after();
-                            const uint64_t a_k = a_desc0 + static_cast<uint64_t>((2 * ks * kAChunkBytes) >> 4);
                             const uint64_t b_k = b_desc0 + static_cast<uint64_t>((w2.slot * kW2StageBytes) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < kKSlice / 16; ++kk) {
-                                const uint64_t a_desc =
-                                    a_k + static_cast<uint64_t>(((kk >> 2) * kAChunkBytes + (kk & 3) * 32) >> 4);
+                                // K elements ks*128 + 16 kk .. + 15: 8 TMEM columns of A
+                                const uint32_t a_tmem =
+                                    tmem + kACol + static_cast<uint32_t>((ks * kKSlice + 16 * kk) >> 1);
                                 const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
-                                umma_bf16_pair(d_tmem, a_desc, b_desc, idesc, (ks | kk) ? 1u : 0u);
+                                umma_bf16_pair_ts(d_tmem, a_tmem, b_desc, idesc, (ks | kk) ? 1u : 0u);
                             }
                             issued_any = true;
                             umma_commit_pair_mask(bar_w2_empty + 8 * w2.slot, both);
@@ -422,7 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (!ok) break;
                         umma_commit_pair_mask(bar_tfull + 8 * acc.slot, both);
-                        acc.next(kAcc);
+                        PAIR_TRACE(k, ps, j, 4);
+                        acc.next(kPairAcc);
                     }
                     if (!ok) break;
                     umma_commit_pair_mask(bar_aempty, both);
@@ -457,27 +481,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_sync512();
 
-        // this warp's share of the A gather of pass ps: rows 8 warp .. + 7, lane l copies 8
-        // of the 32 16-byte pieces of row 8 warp + l/4 (zeros for rows without a request)
+        // this warp's share of A for pass ps: K elements 64c .. 64c + 63 of the W1 rows of
+        // its quadrant's 32 requests (zeros for rows without a request), loaded into
+        // registers (a whole 128-byte line per lane) and stored into the A columns of TMEM
         auto gather = [&](int ps) {
-            const int r = 8 * warp + (lane >> 2);
-            const int tok = sh.tok[ps][r];
+            const int tok = sh.tok[ps][row];
+            uint32_t v[32];
+            if (tok >= 0) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.W1 + static_cast<size_t>(tok) * kRank + c * 64);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int unit = (lane & 3) * 8 + i;                 // 16-byte piece of the row
-                const uint32_t dst = sA + (unit >> 3) * kAChunkBytes + r * 128 +
-                                     (((unit & 7) ^ (r & 7)) << 4);
-                if (tok >= 0)
-                    cp_async_16(dst, p.W1 + static_cast<size_t>(tok) * kRank + unit * 8);
-                else
-                    sts128_zero(dst);
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 t = __ldg(src + i);
+                    v[4 * i] = t.x;
+                    v[4 * i + 1] = t.y;
+                    v[4 * i + 2] = t.z;
+                    v[4 * i + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0u;
             }
-            cp_async_wait_all();
-            fence_proxy_async_smem();
+            tmem_st_32x32b_x32(t_lane + kACol + static_cast<uint32_t>(c * 32), v);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 if (lead) mbar_arrive(bar_afull);
-                else mbar_arrive_cluster(afull_lead);
+                else mbar_arrive_remote(afull_lead);
             }
             ++a_count;
         };
@@ -515,11 +546,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         for (int k = 1; k <= p.gamma; ++k) {
             if (ok) {
-                // L2 prefetch of the W1 rows of the later passes of this position (4 lines a row)
-                const int r = 8 * warp + (lane >> 2);
+                // L2 prefetch of the W1 lines the later passes of this position will gather
                 for (int ps = 1; ps < npass; ++ps) {
-                    const int tok = sh.tok[ps][r];
-                    if (tok >= 0) prefetch_l2(p.W1 + static_cast<size_t>(tok) * kRank + (lane & 3) * 64);
+                    const int tok = sh.tok[ps][row];
+                    if (tok >= 0) prefetch_l2(p.W1 + static_cast<size_t>(tok) * kRank + c * 64);
                 }
                 if (__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty, (a_count & 1u) ^ 1u, ctl, p)))
                     gather(0);
@@ -544,11 +574,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (ok && !__all_sync(0xFFFFFFFFu,
                                           wait_bar(bar_tfull + 8 * acc.slot, acc.phase, ctl, p)))
                         ok = false;
+                    if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 16 + (warp == 12) * 4);
                     if (ok && box < nbox) {
                         tc_fence_after();
                         Ring my = ur;
                         for (int i = 0; i < box; ++i) my.next(kUSlots);
                         if (__all_sync(0xFFFFFFFFu, wait_bar(bar_u_full + 8 * my.slot, my.phase, ctl, p))) {
+                            if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 17 + (warp == 12) * 4);
                             if (active && c < count) {
                                 uint32_t a[32];
                                 tmem_ld_32x32b_x32(
@@ -563,16 +595,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                         }
                     }
+                    if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 18 + (warp == 12) * 4);
                     for (int i = 0; i < nbox; ++i) ur.next(kUSlots);
                     if (ok) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
                             if (lead) mbar_arrive(bar_tempty + 8 * acc.slot);
-                            else mbar_arrive_cluster(tempty_lead + 8 * acc.slot);
+                            else mbar_arrive_remote(tempty_lead + 8 * acc.slot);
                         }
                     }
-                    acc.next(kAcc);
+                    acc.next(kPairAcc);
                     // the next pass's rows are gathered as soon as the MMAs have released A
                     if (ok && !next_gathered &&
                         __all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty, (a_count & 1u) ^ 1u))) {
