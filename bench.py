@@ -68,13 +68,20 @@ def _kernel_sha():
     return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
-def _traffic_per_launch(workload_name):
-    """DRAM bytes per draft launch from the committed ncu summary, if the kernel is unchanged."""
+def _traffic_per_launch(workload_name, gamma):
+    """DRAM bytes per draft launch from the committed ncu summary, if the kernel is unchanged.
+
+    Each entry names the workload and the draft length it stands for; an entry captured at a
+    shorter draft length than the launch it stands for carries its bytes already scaled by
+    the positions (its ``captured_gamma`` says so)."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        if t.get("kernel_sha") == _kernel_sha() and t.get("workload") == workload_name:
-            return float(t["dram_bytes_per_launch"])
+        if t.get("kernel_sha") != _kernel_sha():
+            return None
+        for e in t.get("entries", []):
+            if e.get("workload") == workload_name and int(e.get("gamma", -1)) == gamma:
+                return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -359,6 +366,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3-8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--gamma", type=int, default=None,
+                    help="draft length instead of the workload's own (e.g. a short case to profile)")
     ap.add_argument("--ref-sample", type=int, default=4)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--eager", action="store_true", help="launch kernels one by one (no CUDA graph)")
@@ -371,6 +380,9 @@ def main():
                          "steps earlier, on a side stream that overlaps the draft kernel")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
+    if args.gamma is not None:
+        import re
+        wl = wl.with_(gamma=args.gamma, name=re.sub(r"gamma=\d+", f"gamma={args.gamma}", wl.name))
     if args.stage == "sts-fit":
         if int(os.environ.get("RANK", "0")) == 0 and args.impl == "ours":
             run_sts_fit(args)
@@ -651,7 +663,7 @@ def main():
         t_tc = flops / (tflops * 1e12)
         roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "achieved": achieved,
                 "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
-                "traffic": None if rnn else _traffic_per_launch(wl.name),
+                "traffic": None if rnn else _traffic_per_launch(wl.name, gamma),
                 "kernel": ("markov_pair_kernel" if B > 128 and not rnn else "markov_draft_kernel")
                 + (" + confidence head" if fused else ""),
                 "kernel_ms": draft_mean, "algorithmic_bytes": algo_bytes,

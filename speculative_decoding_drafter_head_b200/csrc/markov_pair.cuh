@@ -21,10 +21,10 @@
 // Per CTA: 16 epilogue warps (four per TMEM lane quadrant, one 32-column chunk of every
 // tile each), warp 16 the W2 producer (TMA, 64 columns x 128 K rows per stage), warp 17
 // the U producer (TMA, 128 rows x 64 columns per box), warp 18 the MMA issuer in the even
-// CTA and, in the odd CTA, the relay that tells the even CTA when the odd CTA's W2 stage
-// has landed.  Signals that cross the pair: the odd CTA's W2 arrivals (relayed), its A
-// gathers and its accumulator releases arrive on the even CTA's barriers; the even CTA's
-// MMA completions arrive on both CTAs' barriers through one pair commit.
+// CTA.  Signals that cross the pair: the odd CTA's W2 copies complete on the even CTA's
+// stage barrier (.cta_group::2 copies; the even CTA arms it for both halves), and its A
+// gathers and accumulator releases arrive on the even CTA's barriers; the even CTA's MMA
+// completions arrive on both CTAs' barriers through one pair commit.
 //
 // Selection as in markov_draft_kernel: greedy argmax with the smallest index on ties, or
 // Gumbel-max with Philox noise keyed (seed, request, position, vocabulary index).  Here the
@@ -62,8 +62,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGumbel2Max = 24.0f;
 
 struct Ctl {
-    unsigned long long w2_full[kW2Stages];   // this CTA's W2 stage has landed (local TMA)
-    unsigned long long w2_peer[kW2Stages];   // even CTA: the odd CTA's stage has landed
+    unsigned long long w2_full[kW2Stages];   // even CTA: both CTAs' W2 halves have landed
     unsigned long long w2_empty[kW2Stages];  // both: the pair MMAs have read the stage
     unsigned long long u_full[kUSlots];
     unsigned long long u_empty[kUSlots];
@@ -110,18 +109,17 @@ __device__ __forceinline__ void give_up(Ctl &ctl, const Params &p, unsigned code
     atomicExch(p.abort_flag, 1u);
 }
 
-// Bounded wait on an mbarrier phase; `cluster` selects acquire at cluster scope (for
-// barriers that the other CTA of the pair arrives on).  False once this CTA or any other
-// gave up, or the wait ran out.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl &ctl, const Params &p,
-                                         bool cluster = false)
+// Bounded wait on an mbarrier phase.  CTA-scope acquire also for the barriers that the
+// other CTA of the pair arrives on: what those arrivals order is tensor-core work (A
+// stores, accumulator reads, TMA landings), which the tcgen05 fences around the arrive and
+// the wait order (the pairing CUTLASS's two-SM pipelines use too).  False once this CTA or
+// any other gave up, or the wait ran out.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl &ctl, const Params &p)
 {
-    if (cluster ? mbar_try_wait_cluster(bar, parity, 0) : mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-        if (cluster ? mbar_try_wait_cluster(bar, parity, kWaitHintNs)
-                    : mbar_try_wait_sleep(bar, parity, kWaitHintNs))
-            return true;
+        if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
         if (*reinterpret_cast<volatile int *>(&ctl.abort) ||
             *reinterpret_cast<volatile unsigned int *>(p.abort_flag)) {
             *reinterpret_cast<volatile int *>(&ctl.abort) = 1;
@@ -132,6 +130,24 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Ctl &ctl
             return false;
         }
     }
+}
+
+// Wait for the last use of every slot of a ring after `issued` uses in total.  If the
+// kernel is aborting, a stage may never be used or completed: then the copies this CTA may
+// still have in flight get a fixed time to land, and the result is false.
+constexpr uint64_t kSettleNs = 200000;
+__device__ __forceinline__ bool drain_or_settle(uint32_t bar0, int n, long long issued, Ctl &ctl,
+                                                const Params &p)
+{
+    for (int s = 0; s < n; ++s) {
+        const long long uses = issued / n + (s < issued % n ? 1 : 0);
+        if (uses > 0 && !wait_bar(bar0 + 8 * s, static_cast<uint32_t>((uses - 1) & 1), ctl, p)) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < kSettleNs) __nanosleep(1000);
+            return false;
+        }
+    }
+    return true;
 }
 
 // The j-th tile of pass `pass`: forward on even passes, backward on odd ones.
@@ -266,7 +282,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int npass = (p.B + kPairRows - 1) / kPairRows;   // 256-request blocks per position
 
     const uint32_t bar_w2_full = smem_u32(&ctl.w2_full[0]);
-    const uint32_t bar_w2_peer = smem_u32(&ctl.w2_peer[0]);
     const uint32_t bar_w2_empty = smem_u32(&ctl.w2_empty[0]);
     const uint32_t bar_u_full = smem_u32(&ctl.u_full[0]);
     const uint32_t bar_u_empty = smem_u32(&ctl.u_empty[0]);
@@ -279,7 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kW2Stages; ++s) {
             mbar_init(bar_w2_full + 8 * s, 1);
-            mbar_init(bar_w2_peer + 8 * s, 1);
             mbar_init(bar_w2_empty + 8 * s, 1);
         }
         for (int s = 0; s < kUSlots; ++s) {
@@ -313,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ W2 producer (both CTAs)
         if (lane == 0) {
             const uint64_t pol_w2 = l2_policy_evict_last();
+            const uint32_t w2_full_lead = mapa_shared(bar_w2_full, 0);
             Ring w2;
             long long issued = 0;
             bool ok = true;
@@ -330,18 +345,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 break;
                             }
                             PAIR_TRACE(k, ps, j, 8 + ks);
+                            // both halves count on the even CTA's barrier, armed there for both
                             const uint32_t bar = bar_w2_full + 8 * w2.slot;
-                            mbar_arrive_expect_tx(bar, kW2StageBytes);
-                            tma_load_2d(sW2 + w2.slot * kW2StageBytes, &tm_w2, bar, x, ks * kKSlice,
-                                        pol_w2);
+                            if (lead) {
+                                mbar_arrive_expect_tx(bar, 2 * kW2StageBytes);
+                                tma_load_2d(sW2 + w2.slot * kW2StageBytes, &tm_w2, bar, x,
+                                            ks * kKSlice, pol_w2);
+                            } else {
+                                tma_load_2d_pair(sW2 + w2.slot * kW2StageBytes, &tm_w2, w2_full_lead + 8 * w2.slot,
+                                                 x, ks * kKSlice, pol_w2);
+                            }
                             ++issued;
                             w2.next(kW2Stages);
                         }
                     }
                 }
-            // this CTA's copies land before exit; the last pair commits on w2_empty too
-            drain_ring(bar_w2_full, kW2Stages, issued, p);
-            drain_ring(bar_w2_empty, kW2Stages, issued, p);
+            // the copies land before exit: the even CTA sees both halves on w2_full, and every
+            // stage the MMAs released (w2_empty, in both CTAs) had landed
+            if (!lead || drain_or_settle(bar_w2_full, kW2Stages, issued, ctl, p))
+                drain_or_settle(bar_w2_empty, kW2Stages, issued, ctl, p);
         }
     } else if (warp == kWarpU) {
         // ------------------------------------------------------------ U producer (both CTAs)
@@ -376,24 +398,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             drain_ring(bar_u_full, kUSlots, issued, p);
         }
     } else if (warp == kWarpMma) {
+#ifdef DSPARK_TRACE
         if (lane == 0 && !lead) {
-            // -------------------------------------------------------- relay (odd CTA)
-            // tell the even CTA when each of this CTA's W2 stages has landed
-            const uint32_t peer_bar0 = mapa_shared(bar_w2_peer, 0);
-            Ring w2;
-            bool ok = true;
-            for (int k = 1; k <= p.gamma && ok; ++k)
-                for (int ps = 0; ps < npass && ok; ++ps)
-                    for (int j = 0; j < ntiles * kKSlices && ok; ++j) {
-                        if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
-                            ok = false;
-                            break;
-                        }
-                        PAIR_TRACE(k, ps, j / kKSlices, 12 + (j & 1));
-                        mbar_arrive_remote(peer_bar0 + 8 * w2.slot);
-                        w2.next(kW2Stages);
+            // trace only: when each accumulator of positions 1-2 completes, by polling
+            Ring acc;
+            bool live = true;
+            for (int k = 1; k <= 2 && k <= p.gamma && live; ++k)
+                for (int ps = 0; ps < npass && live; ++ps)
+                    for (int j = 0; j < ntiles && live; ++j) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (!mbar_test_wait(bar_tfull + 8 * acc.slot, acc.phase))
+                            if (globaltimer_ns() - t0 > p.timeout_ns) {
+                                live = false;
+                                break;
+                            }
+                        PAIR_TRACE(k, ps, j, 5);
+                        acc.next(kPairAcc);
                     }
-        } else if (lane == 0) {
+        }
+#endif
+        if (lane == 0 && lead) {
             // -------------------------------------------------------- pair MMA issuer (even CTA)
             Ring w2, acc;
             const uint64_t b_desc0 = smem_desc(sW2, kW2StageBytes, 1024, kSwizzle128B);
@@ -404,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 1; k <= p.gamma && ok; ++k)
                 for (int ps = 0; ps < npass && ok; ++ps) {
                     const int pass = (k - 1) * npass + ps;
-                    if (!wait_bar(bar_afull, a_count & 1u, ctl, p, true)) {
+                    if (!wait_bar(bar_afull, a_count & 1u, ctl, p)) {
                         ok = false;
                         break;
                     }
@@ -415,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(kPairRows),
                                                               static_cast<uint32_t>(count * kUnit), 1);
                         PAIR_TRACE(k, ps, j, 0);
-                        if (!wait_bar(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p, true)) {
+                        if (!wait_bar(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p)) {
                             ok = false;
                             break;
                         }
@@ -423,8 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
                         for (int ks = 0; ks < kKSlices; ++ks) {
-                            if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p) ||
-                                !wait_bar(bar_w2_peer + 8 * w2.slot, w2.phase, ctl, p, true)) {
+                            if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
                                 ok = false;
                                 break;
                             }
@@ -570,41 +593,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
                     const int nbox = (count + 1) >> 1;
                     const int box = c >> 1;
+                    // the U box first (it is usually there already), then the accumulator: the
+                    // chunk goes to registers and the slot is released at once, so that the
+                    // next MMAs into it overlap the arithmetic below
+                    Ring my = ur;
+                    for (int i = 0; i < box; ++i) my.next(kUSlots);
+                    const bool has_box = box < nbox;
+                    if (ok && has_box &&
+                        !__all_sync(0xFFFFFFFFu, wait_bar(bar_u_full + 8 * my.slot, my.phase, ctl, p)))
+                        ok = false;
+                    if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 12 + (warp == 12));
                     // warp-uniform: tcgen05.ld below needs every lane of the warp
                     if (ok && !__all_sync(0xFFFFFFFFu,
                                           wait_bar(bar_tfull + 8 * acc.slot, acc.phase, ctl, p)))
                         ok = false;
                     if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 16 + (warp == 12) * 4);
-                    if (ok && box < nbox) {
-                        tc_fence_after();
-                        Ring my = ur;
-                        for (int i = 0; i < box; ++i) my.next(kUSlots);
-                        if (__all_sync(0xFFFFFFFFu, wait_bar(bar_u_full + 8 * my.slot, my.phase, ctl, p))) {
-                            if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 17 + (warp == 12) * 4);
-                            if (active && c < count) {
-                                uint32_t a[32];
-                                tmem_ld_32x32b_x32(
-                                    t_lane + static_cast<uint32_t>(acc.slot * kAccCols + c * kUnit), a);
-                                tmem_wait_ld();
-                                chunk_update(best, a, sU + my.slot * kUSlotBytes, row, c & 1,
-                                             (u_begin + first + c) * kUnit, p, rn, c2);
-                            }
+                    if (ok) {
+                        auto release = [&]() {
+                            tc_fence_before();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(bar_u_empty + 8 * my.slot);
+                            if (lane == 0) {
+                                if (lead) mbar_arrive(bar_tempty + 8 * acc.slot);
+                                else mbar_arrive_remote(tempty_lead + 8 * acc.slot);
+                            }
+                        };
+                        tc_fence_after();
+                        if (active && c < count) {
+                            uint32_t a[32];
+                            tmem_ld_32x32b_x32(
+                                t_lane + static_cast<uint32_t>(acc.slot * kAccCols + c * kUnit), a);
+                            tmem_wait_ld();
+                            release();
+                            if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 17 + (warp == 12) * 4);
+                            chunk_update(best, a, sU + my.slot * kUSlotBytes, row, c & 1,
+                                         (u_begin + first + c) * kUnit, p, rn, c2);
                         } else {
-                            ok = false;
+                            release();
                         }
+                        __syncwarp();
+                        if (lane == 0 && has_box) mbar_arrive(bar_u_empty + 8 * my.slot);
                     }
                     if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 18 + (warp == 12) * 4);
                     for (int i = 0; i < nbox; ++i) ur.next(kUSlots);
-                    if (ok) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (lead) mbar_arrive(bar_tempty + 8 * acc.slot);
-                            else mbar_arrive_remote(tempty_lead + 8 * acc.slot);
-                        }
-                    }
                     acc.next(kPairAcc);
                     // the next pass's rows are gathered as soon as the MMAs have released A
                     if (ok && !next_gathered &&

@@ -153,6 +153,19 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *desc, uint
         : "memory");
 }
 
+// 2D tile load into this CTA's shared memory whose completion is counted on an mbarrier
+// of either CTA of the pair (.cta_group::2): `bar` is a shared::cluster address, e.g. the
+// even CTA's barrier through mapa.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *desc, uint32_t bar,
+                                                 int c0, int c1, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(desc)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 // TMEM allocation: executed by one whole warp; the TMEM address lands in smem.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
@@ -278,22 +291,6 @@ __device__ __forceinline__ void cluster_sync()
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar)
 {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-
-// try_wait with acquire at cluster scope: for barriers that other CTAs of the cluster
-// arrive on, so that their writes before the arrival are visible after the wait.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity,
-                                                      uint32_t hint_ns)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
 }
 
 // TMEM allocation for a CTA pair: one warp of each CTA (same warp index in both) runs
