@@ -40,8 +40,7 @@ import synth  # noqa: E402
 PARITY_MACS = 3.5e11          # oracle multiply-adds spent on the bench line's parity check
 METRIC = "draft tokens/s (Markov head+confidence+schedule+verify); % of HBM/TC roofline"
 UNIT = "tokens/s"
-DRAFT_SRCS = [os.path.join(ROOT, "speculative_decoding_drafter_head_b200", "csrc", f)
-              for f in ("markov_draft.cuh", "markov_pair.cuh")]
+CSRC = os.path.join(ROOT, "speculative_decoding_drafter_head_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "markov_draft_traffic.json")
 
 
@@ -54,13 +53,13 @@ def _peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def _kernel_sha():
-    """Hash of the draft kernel's source with comments and blank space removed, so that the
+def _kernel_sha(sources):
+    """Hash of a kernel's source files with comments and blank space removed, so that a
     committed DRAM-traffic figure stays attached to the code it was measured on."""
     import re
     src = ""
-    for path in DRAFT_SRCS:
-        with open(path, encoding="utf-8") as f:
+    for name in sources:
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
             src += f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
@@ -71,16 +70,15 @@ def _kernel_sha():
 def _traffic_per_launch(workload_name, gamma):
     """DRAM bytes per draft launch from the committed ncu summary, if the kernel is unchanged.
 
-    Each entry names the workload and the draft length it stands for; an entry captured at a
-    shorter draft length than the launch it stands for carries its bytes already scaled by
-    the positions (its ``captured_gamma`` says so)."""
+    Each entry names the workload and draft length it stands for and the source files of
+    the kernel it was measured on, with their hash; an entry whose files have changed
+    since is ignored."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        if t.get("kernel_sha") != _kernel_sha():
-            return None
         for e in t.get("entries", []):
-            if e.get("workload") == workload_name and int(e.get("gamma", -1)) == gamma:
+            if (e.get("workload") == workload_name and int(e.get("gamma", -1)) == gamma
+                    and e.get("kernel_sha") == _kernel_sha(e["sources"])):
                 return float(e["dram_bytes_per_launch"])
     except Exception:
         pass

@@ -41,7 +41,11 @@ typedef enum {
     DSPARK_NOT_MONOTONE = 4,      /* device: scores increase along a request      */
     DSPARK_CUDA_ERROR = 5,        /* a CUDA runtime/driver call failed            */
     DSPARK_TIMEOUT = 6,           /* device: a bounded wait ran out               */
-    DSPARK_INVALID_TOKEN = 7      /* device: a token id or length out of range    */
+    DSPARK_INVALID_TOKEN = 7,     /* device: a token id or length out of range    */
+    DSPARK_BAD_LAUNCH = 8         /* device: a kernel found itself launched in a
+                                     shape it cannot run in (e.g. a tool re-issued
+                                     the launch without its thread-block cluster);
+                                     it returned before touching memory          */
 } dspark_status;
 
 /* Text for a status code (static storage). */

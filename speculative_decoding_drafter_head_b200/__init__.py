@@ -31,6 +31,7 @@ __all__ = [
 STATUS = {
     0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "WORKSPACE_TOO_SMALL",
     4: "NOT_MONOTONE", 5: "CUDA_ERROR", 6: "TIMEOUT", 7: "INVALID_TOKEN",
+    8: "BAD_LAUNCH",
 }
 
 EXPORTED = (

@@ -161,6 +161,7 @@ const char *dspark_status_string(int status)
     case DSPARK_CUDA_ERROR: return "CUDA error";
     case DSPARK_TIMEOUT: return "device wait timed out";
     case DSPARK_INVALID_TOKEN: return "token id or verify length out of range";
+    case DSPARK_BAD_LAUNCH: return "kernel launched in a shape it cannot run in";
     default: return "unknown status";
     }
 }
@@ -265,7 +266,7 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     // device reset
     const bool fused = conf && !pair;    // the pair kernel leaves confidence to its own launch
     void (*kern)(const CUtensorMap, const CUtensorMap, const D::Params) =
-        pair ? D::pairk::markov_pair_kernel
+        pair ? (mode ? D::pairk::markov_pair_kernel<true> : D::pairk::markov_pair_kernel<false>)
         : Whh ? (M == 64 ? D::markov_draft_kernel<64, true> : D::markov_draft_kernel<128, true>)
         : fused ? (M == 64 ? D::markov_draft_kernel<64, false, true>
                            : D::markov_draft_kernel<128, false, true>)
@@ -285,10 +286,10 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          D::kDynSmem) != cudaSuccess)
                     return DSPARK_CUDA_ERROR;
-            if (cudaFuncSetAttribute(D::pairk::markov_pair_kernel,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     D::pairk::kDynSmem) != cudaSuccess)
-                return DSPARK_CUDA_ERROR;
+            for (auto f : {D::pairk::markov_pair_kernel<false>, D::pairk::markov_pair_kernel<true>})
+                if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         D::pairk::kDynSmem) != cudaSuccess)
+                    return DSPARK_CUDA_ERROR;
             dev->pair_clusters = 0;
             dev->draft_ctx = ctx;
         }
@@ -305,6 +306,10 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     prm.inv_tau = mode == 1 ? 1.0f / temperature : 1.0f;
     prm.seed_lo = static_cast<uint32_t>(seed);
     prm.seed_hi = static_cast<uint32_t>(seed >> 32);
+    for (int r = 0; r < 10; ++r) {   // the Philox key schedule (Weyl increments), once per launch
+        prm.rk0[r] = prm.seed_lo + static_cast<uint32_t>(r) * 0x9E3779B9u;
+        prm.rk1[r] = prm.seed_hi + static_cast<uint32_t>(r) * 0xBB67AE85u;
+    }
     prm.b_offset = b_offset;
     prm.x_out = x_out;
     prm.logit_out = logit_x_out;

@@ -74,6 +74,7 @@ struct Params {
     int B, gamma, V, mode;
     float inv_tau;
     uint32_t seed_lo, seed_hi;
+    uint32_t rk0[10], rk1[10];   // Philox round keys: (seed_lo + r W0, seed_hi + r W1), r = 0..9
     int b_offset;
     int32_t *x_out;
     float *logit_out;

@@ -178,22 +178,31 @@ __device__ __forceinline__ RowNoise row_noise(uint32_t y, uint32_t z, uint32_t k
     return n;
 }
 
-__device__ __forceinline__ uint4 philox_row(uint32_t x, const RowNoise &n, uint32_t k0,
-                                            uint32_t k1)
+// hi and lo halves of a 32 x 32-bit product from one wide multiply
+__device__ __forceinline__ void mul_wide(uint32_t a, uint32_t b, uint32_t &hi, uint32_t &lo)
 {
-    const uint32_t hi0 = __umulhi(kPhM0, x), lo0 = kPhM0 * x;    // round 1
-    const uint32_t cz = hi0 ^ k1;
-    k0 += kPhW0;
-    k1 += kPhW1;
-    const uint32_t hi1 = __umulhi(kPhM1, cz), lo1 = kPhM1 * cz;   // round 2
-    uint4 c = make_uint4(hi1 ^ n.l1 ^ k0, lo1, n.h0p ^ lo0 ^ k1, n.l0p);
+    uint64_t r;
+    asm("mul.wide.u32 %0, %1, %2;" : "=l"(r) : "r"(a), "r"(b));
+    hi = static_cast<uint32_t>(r >> 32);
+    lo = static_cast<uint32_t>(r);
+}
+
+// Philox4x32-10 of the counter (x, y, z, 0) for the row `n` describes.  The round keys
+// come precomputed from the launch parameters (constant memory), so that no round spends
+// instructions on the key schedule, and each round's two products are wide multiplies.
+__device__ __forceinline__ uint4 philox_row(uint32_t x, const RowNoise &n, const Params &p)
+{
+    uint32_t hi0, lo0, hi1, lo1;
+    mul_wide(kPhM0, x, hi0, lo0);                                 // round 1
+    const uint32_t cz = hi0 ^ p.rk1[0];
+    mul_wide(kPhM1, cz, hi1, lo1);                                // round 2
+    uint4 c = make_uint4(hi1 ^ n.l1 ^ p.rk0[1], lo1, n.h0p ^ lo0 ^ p.rk1[1], n.l0p);
 #pragma unroll
     for (int round = 2; round < 10; ++round) {
-        k0 += kPhW0;
-        k1 += kPhW1;
-        const uint32_t a0 = __umulhi(kPhM0, c.x), b0 = kPhM0 * c.x;
-        const uint32_t a1 = __umulhi(kPhM1, c.z), b1 = kPhM1 * c.z;
-        c = make_uint4(a1 ^ c.y ^ k0, b1, a0 ^ c.w ^ k1, b0);
+        uint32_t a0, b0, a1, b1;
+        mul_wide(kPhM0, c.x, a0, b0);
+        mul_wide(kPhM1, c.z, a1, b1);
+        c = make_uint4(a1 ^ c.y ^ p.rk0[round], b1, a0 ^ c.w ^ p.rk1[round], b0);
     }
     return c;
 }
@@ -215,7 +224,9 @@ __device__ __forceinline__ float gumbel2_from_word(uint32_t w)
 
 // One 32-column chunk of one request row: l = acc + U; greedy keeps the largest logit,
 // Gumbel-max the largest l c2 + noise (c2 = log2(e)/tau); strict improvement keeps the
-// smallest column on ties.
+// smallest column on ties.  Greedy and Gumbel are separate kernel instances (kGumbel), so
+// that the greedy one carries none of the noise code.
+template <bool kGumbel>
 __device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[32], uint32_t sU,
                                              int row, int h, int v0, const Params &p,
                                              const RowNoise &rn, float c2)
@@ -227,7 +238,7 @@ __device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[
         for (int i = 0; i < 32; ++i)
             if (v0 + i >= p.V) l[i] = -INFINITY;
     }
-    if (p.mode == 0) {
+    if constexpr (!kGumbel) {
         const float mx = max32(l);
         if (mx > best.s) {
             best.v = static_cast<uint32_t>(v0 + first_index(l, mx));
@@ -242,7 +253,7 @@ __device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[
     float s[32];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-        const uint4 w = philox_row(static_cast<uint32_t>((v0 >> 2) + q), rn, p.seed_lo, p.seed_hi);
+        const uint4 w = philox_row(static_cast<uint32_t>((v0 >> 2) + q), rn, p);
         s[4 * q + 0] = fmaf(l[4 * q + 0], c2, gumbel2_from_word(w.x));
         s[4 * q + 1] = fmaf(l[4 * q + 1], c2, gumbel2_from_word(w.y));
         s[4 * q + 2] = fmaf(l[4 * q + 2], c2, gumbel2_from_word(w.z));
@@ -257,6 +268,7 @@ __device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[
     }
 }
 
+template <bool kGumbel>
 __global__ void __launch_bounds__(kThreads, 1)
     markov_pair_kernel(const __grid_constant__ CUtensorMap tm_w2,
                        const __grid_constant__ CUtensorMap tm_u, const Params p)
@@ -265,6 +277,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ Shared sh;
     Ctl &ctl = sh.ctl;
 
+    // everything below assumes clusters of exactly two CTAs and whole pairs: a launch in
+    // any other shape (a tool re-issuing it without the cluster, say) stops here, before
+    // any pair instruction or cross-CTA access
+    if (cluster_nctarank() != 2u || (gridDim.x & 1u) || blockDim.x != kThreads) {
+        if (threadIdx.x == 0) record_error(DSPARK_BAD_LAUNCH);
+        return;
+    }
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();          // 0: even CTA (issues the MMAs)
@@ -444,16 +463,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         PAIR_TRACE(k, ps, j, 1);
+                        static_assert(kKSlices == 2, "a tile's K is two W2 stages");
+                        // both K halves are waited for up front, so that the tile's 16 MMAs
+                        // issue back to back: the tensor core's queue is short, and a wait
+                        // between them leaves it idle
+                        Ring w2b = w2;
+                        w2b.next(kW2Stages);
+                        if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p) ||
+                            !wait_bar(bar_w2_full + 8 * w2b.slot, w2b.phase, ctl, p)) {
+                            ok = false;
+                            break;
+                        }
+                        PAIR_TRACE(k, ps, j, 2);
                         tc_fence_after();
                         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
+#pragma unroll
                         for (int ks = 0; ks < kKSlices; ++ks) {
-                            if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p)) {
-                                ok = false;
-                                break;
-                            }
-                            PAIR_TRACE(k, ps, j, 2 + ks);
-                            tc_fence_after();
-                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((w2.slot * kW2StageBytes) >> 4);
+                            const uint32_t slot = ks ? w2b.slot : w2.slot;
+                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((slot * kW2StageBytes) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < kKSlice / 16; ++kk) {
                                 // K elements ks*128 + 16 kk .. + 15: 8 TMEM columns of A
@@ -462,11 +489,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
                                 umma_bf16_pair_ts(d_tmem, a_tmem, b_desc, idesc, (ks | kk) ? 1u : 0u);
                             }
-                            issued_any = true;
-                            umma_commit_pair_mask(bar_w2_empty + 8 * w2.slot, both);
-                            w2.next(kW2Stages);
                         }
-                        if (!ok) break;
+                        issued_any = true;
+                        umma_commit_pair_mask(bar_w2_empty + 8 * w2.slot, both);
+                        umma_commit_pair_mask(bar_w2_empty + 8 * w2b.slot, both);
+                        w2b.next(kW2Stages);
+                        w2 = w2b;
                         umma_commit_pair_mask(bar_tfull + 8 * acc.slot, both);
                         PAIR_TRACE(k, ps, j, 4);
                         acc.next(kPairAcc);
@@ -583,9 +611,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int pass = (k - 1) * npass + ps;
                 const int b_row = ps * kPairRows + static_cast<int>(rank) * kRows + row;
                 const bool active = ps * kPairRows + static_cast<int>(rank) * kRows + q * 32 < p.B;
-                const RowNoise rn = row_noise(static_cast<uint32_t>(k - 1),
-                                              static_cast<uint32_t>(b_row + p.b_offset), p.seed_lo,
-                                              p.seed_hi);
+                const RowNoise rn = kGumbel ? row_noise(static_cast<uint32_t>(k - 1),
+                                                        static_cast<uint32_t>(b_row + p.b_offset),
+                                                        p.seed_lo, p.seed_hi)
+                                            : RowNoise{0u, 0u, 0u, 0u};
                 bool next_gathered = ps + 1 >= npass;
                 RowBest best;
                 for (int j = 0; j < ntiles; ++j) {
@@ -625,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tmem_wait_ld();
                             release();
                             if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 17 + (warp == 12) * 4);
-                            chunk_update(best, a, sU + my.slot * kUSlotBytes, row, c & 1,
+                            chunk_update<kGumbel>(best, a, sU + my.slot * kUSlotBytes, row, c & 1,
                                          (u_begin + first + c) * kUnit, p, rn, c2);
                         } else {
                             release();

@@ -270,6 +270,13 @@ __device__ __forceinline__ uint32_t cluster_ctarank()
     return r;
 }
 
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+    return n;
+}
+
 // Address in CTA `rank` of the cluster that corresponds to this CTA's shared address.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
 {

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     assert ds.status_string(0) == "ok"
-    for code in range(1, 8):
+    for code in range(1, 9):
         assert ds.status_string(code) != "unknown status"
     assert ds.status_string(99) == "unknown status"
 
