@@ -460,7 +460,8 @@ def main():
         lsched = pipeline.LaggedScheduler(B * world, gamma, Tstep, lag=2)
     step_no = [0]
 
-    # the Markov head drafts and scores in one call (one launch for B <= 128); the RNN
+    # the Markov head drafts and scores in one call (one launch, two for Gumbel-max above
+    # 128 requests); the RNN
     # head drafts, then the confidence kernel scores
     fused = not rnn
 
@@ -663,7 +664,8 @@ def main():
                 "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                 "traffic": None if rnn else _traffic_per_launch(wl.name, gamma),
                 "kernel": ("markov_pair_kernel" if B > 128 and not rnn else "markov_draft_kernel")
-                + (" + confidence head" if fused else ""),
+                + ((" + confidence kernel" if wl.mode == 1 and B > 128 else " + confidence head")
+                   if fused else ""),
                 "kernel_ms": draft_mean, "algorithmic_bytes": algo_bytes,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s"}
@@ -689,7 +691,7 @@ def main():
             "parity": parity,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": (3 if fused and B <= 128 else 4) * args.steps,
+            "gpu_launches": (3 if fused and not (wl.mode == 1 and B > 128) else 4) * args.steps,
             "cuda_graph": graph is not None,
             "schedule": "lagged by 2 steps, side stream" if lagged else "this step's scores",
             "head": args.head,

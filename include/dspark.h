@@ -144,12 +144,13 @@ int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x
  *
  * Arguments as for those two calls (U, anchor, W1, W2, mode, temperature, seed, b_offset,
  * x_out, logit_x_out, workspace as for dspark_draft_step; h, w, b_conf, T, d, c_out,
- * P_out as for dspark_confidence_sts), with the same sizes, alignment and errors.  With
- * B <= 128 both run in one launch: one warp of every CTA of the draft kernel computes
- * the hidden-state part of every logit at the start and the rest of each position's
- * scores as soon as the grid barrier of the previous position has fixed x_{k-1}, beside
- * the drafting; the workspace from dspark_workspace_bytes covers it.  With B > 128 the
- * confidence kernel follows as a second launch on the same stream.  c and P agree with
+ * P_out as for dspark_confidence_sts), with the same sizes, alignment and errors.  Both
+ * run in one launch: one warp of every CTA of the draft kernel computes the hidden-state
+ * part of every logit at the start and the rest of each position's scores as soon as the
+ * grid barrier of the previous position has fixed x_{k-1}, beside the drafting; the
+ * workspace from dspark_workspace_bytes covers it.  The exception is Gumbel-max drafting
+ * (mode 1) with B > 128, whose selection arithmetic is the bound: there the confidence
+ * kernel follows as a second launch on the same stream.  c and P agree with
  * dspark_confidence_sts up to the order of the fp32 additions of z.
  */
 int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const void *W1,

@@ -264,9 +264,12 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     // the kernel instance for this call (Markov or RNN head, M = 64 or 128, or the pair
     // kernel); its shared memory limit is set on every call, so nothing cached outlives a
     // device reset
-    const bool fused = conf && !pair;    // the pair kernel leaves confidence to its own launch
+    const bool fused = conf != nullptr;   // the confidence head runs in a warp of the draft kernel
     void (*kern)(const CUtensorMap, const CUtensorMap, const D::Params) =
-        pair ? (mode ? D::pairk::markov_pair_kernel<true> : D::pairk::markov_pair_kernel<false>)
+        pair ? (fused ? (mode ? D::pairk::markov_pair_kernel<true, true>
+                              : D::pairk::markov_pair_kernel<false, true>)
+                      : (mode ? D::pairk::markov_pair_kernel<true, false>
+                              : D::pairk::markov_pair_kernel<false, false>))
         : Whh ? (M == 64 ? D::markov_draft_kernel<64, true> : D::markov_draft_kernel<128, true>)
         : fused ? (M == 64 ? D::markov_draft_kernel<64, false, true>
                            : D::markov_draft_kernel<128, false, true>)
@@ -286,7 +289,10 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          D::kDynSmem) != cudaSuccess)
                     return DSPARK_CUDA_ERROR;
-            for (auto f : {D::pairk::markov_pair_kernel<false>, D::pairk::markov_pair_kernel<true>})
+            for (auto f : {D::pairk::markov_pair_kernel<false, false>,
+                           D::pairk::markov_pair_kernel<true, false>,
+                           D::pairk::markov_pair_kernel<false, true>,
+                           D::pairk::markov_pair_kernel<true, true>})
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          D::pairk::kDynSmem) != cudaSuccess)
                     return DSPARK_CUDA_ERROR;
@@ -367,7 +373,7 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     attr[1].val.clusterDim.x = 2;
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(D::pairk::kThreads);
+    cfg.blockDim = dim3(fused ? D::pairk::kThreadsConfPair : D::pairk::kThreads);
     cfg.gridDim = dim3(dev->sms & ~1);
     cfg.attrs = attr + 1;
     cfg.numAttrs = 1;
@@ -438,11 +444,15 @@ int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const voi
     if (d < 8 || d % 8 != 0 || (d + r) * 2 > 200 * 1024 || gamma > dspark::conf::kMaxGamma)
         return DSPARK_UNSUPPORTED_SHAPE;
     const ConfArgs conf{h, w, b_conf, T, d, c_out, P_out};
+    // Gumbel-max drafting on CTA pairs is bound by its selection arithmetic, and a
+    // confidence warp beside it would take issue slots from it: there the confidence
+    // kernel follows as a second launch instead
+    const bool in_launch = !(mode == 1 && B > 128);
     if (int st = launch_draft(U, anchor, W1, W2, nullptr, B, gamma, V, r, mode, temperature, seed,
                               b_offset, x_out, logit_x_out, workspace, workspace_bytes, stream,
-                              &conf))
+                              in_launch ? &conf : nullptr))
         return st;
-    if (B <= 128) return DSPARK_OK;      // computed inside the draft launch
+    if (in_launch) return DSPARK_OK;     // computed inside the draft launch
     return dspark_confidence_sts(h, anchor, x_out, W1, w, b_conf, T, B, gamma, d, r, V, c_out,
                                  P_out, stream);
 }

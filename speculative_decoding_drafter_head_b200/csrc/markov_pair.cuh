@@ -21,7 +21,7 @@
 // Per CTA: 16 epilogue warps (four per TMEM lane quadrant, one 32-column chunk of every
 // tile each), warp 16 the W2 producer (TMA, 64 columns x 128 K rows per stage), warp 17
 // the U producer (TMA, 128 rows x 64 columns per box), warp 18 the MMA issuer in the even
-// CTA.  Signals that cross the pair: the odd CTA's W2 copies complete on the even CTA's
+// CTA, and in the kConf instances warp 19 the confidence head (as in markov_draft_kernel).  Signals that cross the pair: the odd CTA's W2 copies complete on the even CTA's
 // stage barrier (.cta_group::2 copies; the even CTA arms it for both halves), and its A
 // gathers and accumulator releases arrive on the even CTA's barriers; the even CTA's MMA
 // completions arrive on both CTAs' barriers through one pair commit.
@@ -43,6 +43,8 @@ constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kWarpW2 = kEpiWarps, kWarpU = kEpiWarps + 1, kWarpMma = kEpiWarps + 2;
 constexpr int kThreads = (kEpiWarps + 3) * 32;        // 608
+constexpr int kWarpConfPair = kEpiWarps + 3;          // confidence head (kConf instances)
+constexpr int kThreadsConfPair = kThreads + 32;       // 640
 constexpr int kRows = 128;                            // requests per CTA per pass
 constexpr int kPairRows = 2 * kRows;                  // the pair MMA's M
 constexpr int kW2Stages = 7;
@@ -268,8 +270,8 @@ __device__ __forceinline__ void chunk_update(RowBest &best, const uint32_t (&a)[
     }
 }
 
-template <bool kGumbel>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kGumbel, bool kConf>
+__global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
     markov_pair_kernel(const __grid_constant__ CUtensorMap tm_w2,
                        const __grid_constant__ CUtensorMap tm_u, const Params p)
 {
@@ -280,7 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // everything below assumes clusters of exactly two CTAs and whole pairs: a launch in
     // any other shape (a tool re-issuing it without the cluster, say) stops here, before
     // any pair instruction or cross-CTA access
-    if (cluster_nctarank() != 2u || (gridDim.x & 1u) || blockDim.x != kThreads) {
+    if (cluster_nctarank() != 2u || (gridDim.x & 1u) ||
+        blockDim.x != static_cast<unsigned>(kConf ? kThreadsConfPair : kThreads)) {
         if (threadIdx.x == 0) record_error(DSPARK_BAD_LAUNCH);
         return;
     }
@@ -416,6 +419,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             drain_ring(bar_u_full, kUSlots, issued, p);
         }
+    } else if (kConf && warp == kWarpConfPair) {
+        // ------------------------------------------------------------ confidence head
+        confidence_warp(p, static_cast<int>(gridDim.x));
     } else if (warp == kWarpMma) {
 #ifdef DSPARK_TRACE
         if (lane == 0 && !lead) {

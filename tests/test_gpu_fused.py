@@ -32,6 +32,10 @@ CASES = [
     synth.Workload("fused B=7 V=5000 gumbel", B=7, gamma=12, V=5000, d=256, w_std=0.2,
                    mode=1, tau=0.8, seed=4),
     synth.Workload("fused B=300 V=5000", B=300, gamma=4, V=5000, d=256, w_std=0.2, seed=5),
+    # the pair kernel's confidence warp: Gumbel instance, and three 256-row passes
+    synth.Workload("fused B=260 V=4104 gumbel", B=260, gamma=6, V=4104, d=512, w_std=0.2,
+                   mode=1, tau=0.7, seed=6),
+    synth.Workload("fused B=640 V=2056", B=640, gamma=5, V=2056, d=256, w_std=0.2, seed=7),
 ]
 
 
