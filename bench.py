@@ -4,8 +4,10 @@
 One step = one draft block through the whole path: Markov-head drafting of gamma
 tokens for every request (dspark_draft_step), confidence + STS + survival product
 (dspark_confidence_sts), the prefix scheduler (dspark_schedule_prefix) and strict
-prefix-match verification (dspark_verify_prefix).  The metric is draft tokens per
-second, B * gamma / step time, summed over ranks.
+prefix-match verification (dspark_verify_prefix).  On one GPU with the Markov head the
+step is the single call dspark_step (one launch for B <= 128); with the RNN head, the
+lagged schedule or several ranks it is the calls above in sequence.  The metric is
+draft tokens per second, B * gamma / step time, summed over ranks.
 
     python bench.py [--gpus N --steps K --warmup W] [--workload qwen3-8b]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
@@ -476,9 +478,19 @@ def main():
         if not fused:
             ds.confidence_sts(h, anchor, x, W1, w, wl.b_conf, T, c, P_dst)
 
+    # one process and this step's scores: the whole step is one call (one launch for
+    # B <= 128 and B gamma <= 1024, the calls in sequence above)
+    one_call = fused and world == 1 and not lagged
+
     def step(record=None):
         t = step_no[0]
         step_no[0] += 1
+        if one_call and record is None:
+            ds.step(U, anchor, W1, W2, h, w, wl.b_conf, T, Tstep, target, x, lx, c, P, Lg, Nst,
+                    obj, acc, bonus, ws, mode=wl.mode, temperature=wl.tau, seed=wl.seed,
+                    b_offset=b0)
+            last_L[0] = Lg
+            return
         e0 = e1 = None
         P_dst = lsched.scores(t) if lagged and world == 1 else P
         if record is not None:
@@ -691,8 +703,12 @@ def main():
             "parity": parity,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": (3 if fused and not (wl.mode == 1 and B > 128) else 4) * args.steps,
+            "gpu_launches": ((1 if B <= 128 and B * gamma <= 1024 else 3 if B <= 128 or wl.mode == 0
+                              else 4) if one_call
+                             else (3 if fused and not (wl.mode == 1 and B > 128) else 4))
+                            * args.steps,
             "cuda_graph": graph is not None,
+            "step_call": "dspark_step" if one_call else "separate calls",
             "schedule": "lagged by 2 steps, side stream" if lagged else "this step's scores",
             "head": args.head,
             "clocks": clk,

@@ -161,6 +161,31 @@ int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const voi
                                  size_t workspace_bytes, dspark_stream_t stream);
 
 /*
+ * The whole per-step path in one call: dspark_draft_confidence_step, then
+ * dspark_schedule_prefix on the survival scores it wrote, then dspark_verify_prefix on
+ * the drafts and the lengths.  [G] sections 4-6 and [W] "The Hardware-Aware Prefix
+ * Scheduler"; [S] (strict prefix-match verification with a bonus token).
+ *
+ * Arguments as for those calls (Tstep_us, L_out, N_out, objective_out as for
+ * dspark_schedule_prefix; target, accepted_out, bonus_out as for dspark_verify_prefix),
+ * with their sizes, alignment and errors, and one workspace of dspark_workspace_bytes
+ * bytes for all of it.  With B <= 128 and B gamma <= 1024 it is one launch: after the
+ * last position the draft kernel's CTAs rank every score (one warp per score) and the
+ * last CTA to finish scans, picks N*, writes the lengths and verifies every request,
+ * with the same device code as the two kernels, so the outputs equal those of the
+ * separate calls bit for bit.  Otherwise the calls run as separate launches on the same
+ * stream (there the scheduler kernel's many CTAs are faster than the launch saved).
+ * Outputs are written in stream order; nothing is read back to the host.
+ */
+int dspark_step(const void *U, const int32_t *anchor, const void *W1, const void *W2,
+                const void *h, const void *w, float b_conf, const float *T,
+                const double *Tstep_us, const int32_t *target, int B, int gamma, int V, int r,
+                int d, int mode, float temperature, uint64_t seed, int b_offset, int32_t *x_out,
+                float *logit_x_out, float *c_out, float *P_out, int32_t *L_out, int32_t *N_out,
+                double *objective_out, int32_t *accepted_out, int32_t *bonus_out,
+                void *workspace, size_t workspace_bytes, dspark_stream_t stream);
+
+/*
  * Hardware-aware prefix scheduler: per-request verify lengths that maximise
  * expected accepted tokens per unit time.
  * [W] "The Hardware-Aware Prefix Scheduler" (throughput maximisation against a

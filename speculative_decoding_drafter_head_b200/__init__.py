@@ -23,7 +23,7 @@ from . import _build
 
 __all__ = [
     "DSparkError", "load", "workspace_bytes", "draft_step", "draft_step_rnn",
-    "draft_confidence_step", "confidence_sts", "schedule_prefix",
+    "draft_confidence_step", "step", "confidence_sts", "schedule_prefix",
     "verify_prefix", "sts_fit_workspace_bytes", "sts_fit", "get_error", "status_string", "set_wait_timeout_ns", "debug_barrier_extra",
     "STATUS",
 ]
@@ -39,7 +39,7 @@ EXPORTED = (
     "dspark_confidence_sts", "dspark_schedule_prefix", "dspark_verify_prefix",
     "dspark_get_error", "dspark_set_wait_timeout_ns", "dspark_debug_barrier_extra",
     "dspark_sts_fit_workspace_bytes", "dspark_sts_fit", "dspark_draft_step_rnn",
-    "dspark_draft_confidence_step",
+    "dspark_draft_confidence_step", "dspark_step",
 )
 
 _lib = None
@@ -72,6 +72,8 @@ def load(build_if_missing: bool = True):
     lib.dspark_confidence_sts.argtypes = [p, p, p, p, p, f32, p, i, i, i, i, i, p, p, p]
     lib.dspark_draft_confidence_step.argtypes = [p, p, p, p, p, p, f32, p, i, i, i, i, i, i, f32,
                                                  u64, i, p, p, p, p, p, sz, p]
+    lib.dspark_step.argtypes = [p, p, p, p, p, p, f32, p, p, p, i, i, i, i, i, i, f32, u64, i,
+                                p, p, p, p, p, p, p, p, p, p, sz, p]
     lib.dspark_schedule_prefix.argtypes = [p, i, i, p, p, p, p, p, sz, p]
     lib.dspark_verify_prefix.argtypes = [p, p, p, i, i, p, p, p]
     lib.dspark_sts_fit_workspace_bytes.argtypes = [i, i, i, i]
@@ -168,6 +170,30 @@ def draft_confidence_step(U, anchor, W1, W2, h, w, b_conf: float, T, x_out, logi
         _dev(P_out, torch.float32, "P_out"), _dev(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream))
     _check("dspark_draft_confidence_step", st)
+
+
+def step(U, anchor, W1, W2, h, w, b_conf: float, T, Tstep_us, target, x_out, logit_x_out,
+         c_out, P_out, L_out, N_out, objective_out, accepted_out, bonus_out, workspace,
+         mode: int = 0, temperature: float = 1.0, seed: int = 0, b_offset: int = 0,
+         stream=None):
+    """The whole per-step path in one call (see dspark_step)."""
+    import torch
+    B, gamma, V = U.shape
+    r = W1.shape[1]
+    d = h.shape[2]
+    st = load().dspark_step(
+        _dev(U, torch.bfloat16, "U"), _dev(anchor, torch.int32, "anchor"),
+        _dev(W1, torch.bfloat16, "W1"), _dev(W2, torch.bfloat16, "W2"),
+        _dev(h, torch.bfloat16, "h"), _dev(w, torch.bfloat16, "w"), float(b_conf),
+        _dev(T, torch.float32, "T"), _dev(Tstep_us, torch.float64, "Tstep_us"),
+        _dev(target, torch.int32, "target"), B, gamma, V, r, d, int(mode), float(temperature),
+        int(seed) & (2**64 - 1), int(b_offset), _dev(x_out, torch.int32, "x_out"),
+        _dev(logit_x_out, torch.float32, "logit_x_out"), _dev(c_out, torch.float32, "c_out"),
+        _dev(P_out, torch.float32, "P_out"), _dev(L_out, torch.int32, "L_out"),
+        _dev(N_out, torch.int32, "N_out"), _dev(objective_out, torch.float64, "objective_out"),
+        _dev(accepted_out, torch.int32, "accepted_out"), _dev(bonus_out, torch.int32, "bonus_out"),
+        _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    _check("dspark_step", st)
 
 
 def confidence_sts(h, anchor, x, W1, w, b_conf: float, T, c_out, P_out, stream=None):

@@ -205,12 +205,37 @@ struct ConfArgs {
     float *P_out;
 };
 
+// Inputs and outputs of the scheduler and the verification when they run at the end of
+// the draft launch.
+struct TailArgs {
+    const double *Tstep;
+    const int32_t *target;
+    int32_t *L_out, *N_out;
+    double *objective_out;
+    int32_t *accepted_out, *bonus_out;
+};
+
+// Argument checks of the confidence head when it runs inside the draft launch.
+int check_conf_args(const void *h, const void *w, const float *T, const float *c_out,
+                    const float *P_out, int gamma, int d, int r)
+{
+    if (!h || !w || !T || !c_out || !P_out) return DSPARK_INVALID_ARG;
+    if (!aligned(h, 16) || !aligned(w, 16) || !aligned(T, 4) || !aligned(c_out, 4) ||
+        !aligned(P_out, 4))
+        return DSPARK_INVALID_ARG;
+    if (d < 8 || d % 8 != 0 || (d + r) * 2 > 200 * 1024 || gamma > dspark::conf::kMaxGamma)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    return DSPARK_OK;
+}
+
 // The Markov head (Whh == nullptr) and the RNN head share one kernel and one launcher;
-// with `conf` the Markov head's launch also computes the confidence head.
+// with `conf` the Markov head's launch also computes the confidence head, and with
+// `tail` (B <= 128, with conf) the scheduler and the verification after the last position.
 int launch_draft(const void *U, const int32_t *anchor, const void *W1, const void *W2,
                  const void *Whh, int B, int gamma, int V, int r, int mode, float temperature,
                  uint64_t seed, int b_offset, int32_t *x_out, float *logit_x_out, void *workspace,
-                 size_t workspace_bytes, dspark_stream_t stream, const ConfArgs *conf = nullptr)
+                 size_t workspace_bytes, dspark_stream_t stream, const ConfArgs *conf = nullptr,
+                 const TailArgs *tail = nullptr)
 {
     namespace D = dspark::draft;
     if (!U || !anchor || !W1 || !W2 || !x_out || !logit_x_out || !workspace)
@@ -271,6 +296,8 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
                       : (mode ? D::pairk::markov_pair_kernel<true, false>
                               : D::pairk::markov_pair_kernel<false, false>))
         : Whh ? (M == 64 ? D::markov_draft_kernel<64, true> : D::markov_draft_kernel<128, true>)
+        : (fused && tail) ? (M == 64 ? D::markov_draft_kernel<64, false, true, true>
+                                     : D::markov_draft_kernel<128, false, true, true>)
         : fused ? (M == 64 ? D::markov_draft_kernel<64, false, true>
                            : D::markov_draft_kernel<128, false, true>)
                 : (M == 64 ? D::markov_draft_kernel<64, false> : D::markov_draft_kernel<128, false>);
@@ -284,7 +311,9 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
             void (*const all[])(const CUtensorMap, const CUtensorMap, const D::Params) = {
                 D::markov_draft_kernel<64, false>, D::markov_draft_kernel<128, false>,
                 D::markov_draft_kernel<64, true>, D::markov_draft_kernel<128, true>,
-                D::markov_draft_kernel<64, false, true>, D::markov_draft_kernel<128, false, true>};
+                D::markov_draft_kernel<64, false, true>, D::markov_draft_kernel<128, false, true>,
+                D::markov_draft_kernel<64, false, true, true>,
+                D::markov_draft_kernel<128, false, true, true>};
             for (auto f : all)
                 if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          D::kDynSmem) != cudaSuccess)
@@ -302,7 +331,7 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     }
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    D::Params prm;
+    D::Params prm{};                     // every pointer not set below is null
     prm.anchor = anchor;
     prm.W1 = static_cast<const uint16_t *>(W1);
     prm.B = B;
@@ -347,6 +376,22 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
         prm.P_out = conf->P_out;
         prm.zh = reinterpret_cast<float *>(ws + draft_keys_end(B, gamma));   // the RNN state's space
         prm.zh_done = reinterpret_cast<unsigned int *>(ws + 8);
+    }
+    if (fused && tail && !pair) {
+        // workspace past the argmax keys: zh [B gamma] f32, then rank [B gamma] i32 (the
+        // sorted scores live in the kernel's shared memory)
+        const size_t n = static_cast<size_t>(B) * gamma;
+        uint8_t *w0 = ws + draft_keys_end(B, gamma);
+        prm.conf_done = reinterpret_cast<unsigned int *>(ws + 12);
+        prm.tail_done = reinterpret_cast<unsigned int *>(ws + 16);
+        prm.rank = reinterpret_cast<int32_t *>(w0 + round_up(n * 4, 256));
+        prm.Tstep = tail->Tstep;
+        prm.target = tail->target;
+        prm.L_out = tail->L_out;
+        prm.N_out = tail->N_out;
+        prm.objective_out = tail->objective_out;
+        prm.accepted_out = tail->accepted_out;
+        prm.bonus_out = tail->bonus_out;
     }
 
     if (cudaMemsetAsync(ws, 0, draft_keys_end(B, gamma), stream) != cudaSuccess)
@@ -437,12 +482,7 @@ int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const voi
                                  float *logit_x_out, float *c_out, float *P_out, void *workspace,
                                  size_t workspace_bytes, dspark_stream_t stream)
 {
-    if (!h || !w || !T || !c_out || !P_out) return DSPARK_INVALID_ARG;
-    if (!aligned(h, 16) || !aligned(w, 16) || !aligned(T, 4) || !aligned(c_out, 4) ||
-        !aligned(P_out, 4))
-        return DSPARK_INVALID_ARG;
-    if (d < 8 || d % 8 != 0 || (d + r) * 2 > 200 * 1024 || gamma > dspark::conf::kMaxGamma)
-        return DSPARK_UNSUPPORTED_SHAPE;
+    if (int st = check_conf_args(h, w, T, c_out, P_out, gamma, d, r)) return st;
     const ConfArgs conf{h, w, b_conf, T, d, c_out, P_out};
     // Gumbel-max drafting on CTA pairs is bound by its selection arithmetic, and a
     // confidence warp beside it would take issue slots from it: there the confidence
@@ -455,6 +495,51 @@ int dspark_draft_confidence_step(const void *U, const int32_t *anchor, const voi
     if (in_launch) return DSPARK_OK;     // computed inside the draft launch
     return dspark_confidence_sts(h, anchor, x_out, W1, w, b_conf, T, B, gamma, d, r, V, c_out,
                                  P_out, stream);
+}
+
+// The scheduler's second phase runs on one CTA of the draft launch; above this many
+// scores the separate scheduler kernel (many CTAs for the ranks, a 512-thread scan) is
+// faster than the launch it saves (measured: 1024 scores 6 us faster in one launch,
+// 2048 scores 5 us slower).
+constexpr int kTailMaxScores = 1024;
+
+int dspark_step(const void *U, const int32_t *anchor, const void *W1, const void *W2,
+                const void *h, const void *w, float b_conf, const float *T,
+                const double *Tstep_us, const int32_t *target, int B, int gamma, int V, int r,
+                int d, int mode, float temperature, uint64_t seed, int b_offset, int32_t *x_out,
+                float *logit_x_out, float *c_out, float *P_out, int32_t *L_out, int32_t *N_out,
+                double *objective_out, int32_t *accepted_out, int32_t *bonus_out,
+                void *workspace, size_t workspace_bytes, dspark_stream_t stream)
+{
+    if (!Tstep_us || !target || !L_out || !N_out || !objective_out || !accepted_out ||
+        !bonus_out)
+        return DSPARK_INVALID_ARG;
+    if (!aligned(Tstep_us, 8) || !aligned(target, 4) || !aligned(L_out, 4) ||
+        !aligned(N_out, 4) || !aligned(objective_out, 8) || !aligned(accepted_out, 4) ||
+        !aligned(bonus_out, 4))
+        return DSPARK_INVALID_ARG;
+    if (B < 1 || gamma < 1 || B > 32768 || static_cast<long long>(B) * gamma > 65536)
+        return DSPARK_UNSUPPORTED_SHAPE;
+    if (workspace && workspace_bytes < dspark_workspace_bytes(B, gamma, V, r))
+        return DSPARK_WORKSPACE_TOO_SMALL;
+    if (B <= 128 && B * gamma <= kTailMaxScores) {
+        // one launch: drafting, the confidence head, then the scheduler and verification
+        if (int st = check_conf_args(h, w, T, c_out, P_out, gamma, d, r)) return st;
+        const ConfArgs conf{h, w, b_conf, T, d, c_out, P_out};
+        const TailArgs tail{Tstep_us, target, L_out, N_out, objective_out, accepted_out, bonus_out};
+        return launch_draft(U, anchor, W1, W2, nullptr, B, gamma, V, r, mode, temperature, seed,
+                            b_offset, x_out, logit_x_out, workspace, workspace_bytes, stream,
+                            &conf, &tail);
+    }
+    if (int st = dspark_draft_confidence_step(U, anchor, W1, W2, h, w, b_conf, T, B, gamma, V, r,
+                                              d, mode, temperature, seed, b_offset, x_out,
+                                              logit_x_out, c_out, P_out, workspace,
+                                              workspace_bytes, stream))
+        return st;
+    if (int st = dspark_schedule_prefix(P_out, B, gamma, Tstep_us, L_out, N_out, objective_out,
+                                        workspace, workspace_bytes, stream))
+        return st;
+    return dspark_verify_prefix(x_out, L_out, target, B, gamma, accepted_out, bonus_out, stream);
 }
 
 int dspark_confidence_sts(const void *h, const int32_t *anchor, const int32_t *x, const void *W1,

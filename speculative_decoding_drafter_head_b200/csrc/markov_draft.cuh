@@ -38,6 +38,8 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "schedule_prefix.cuh"
+#include "verify_prefix.cuh"
 
 namespace dspark {
 namespace draft {
@@ -103,6 +105,16 @@ struct Params {
     float *c_out, *P_out;        // [B][gamma]
     float *zh;                   // [B][gamma] workspace: the hidden-state part of z
     unsigned int *zh_done;       // workspace counter: CTAs whose zh share is written
+    unsigned int *conf_done;     // workspace counter: CTAs whose confidence warp is done
+    // scheduler and verification in the same launch (kTail): the global top-N over all
+    // B gamma survival scores and the scan over N, then strict prefix-match verification
+    const double *Tstep;         // [B (gamma + 1) + 1] step time for n verified tokens
+    const int32_t *target;       // [B][gamma + 1]
+    int32_t *L_out, *N_out;      // [B], [1]
+    double *objective_out;       // [1]
+    int32_t *accepted_out, *bonus_out;   // [B]
+    int32_t *rank;               // [B gamma] workspace
+    unsigned int *tail_done;     // workspace counter: CTAs whose ranks are written
 };
 
 struct Ctl {
@@ -575,12 +587,17 @@ __device__ __forceinline__ void confidence_warp(const Params &p, int G)
             }
         }
     }
+    // with the scheduler in the launch, it starts once every CTA's scores are written
+    // (also after a failure: the waiter then sees the abort flag)
+    __syncwarp();
+    if (p.conf_done && lane == 0) red_release_add_u32(p.conf_done, 1u);
 }
 
 // kM is the MMA's M (64 when B <= 64, else 128); p.M equals it.  kRnn selects the RNN
 // head (p.Whh set); the Markov instances carry none of its code.  kConf adds the
-// confidence warp (Markov head only).
-template <int kM, bool kRnn, bool kConf = false>
+// confidence warp (Markov head only), kTail (with kConf) the scheduler and the
+// verification after the last position.
+template <int kM, bool kRnn, bool kConf = false, bool kTail = false>
 __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
     markov_draft_kernel(const __grid_constant__ CUtensorMap tm_w2,
                         const __grid_constant__ CUtensorMap tm_u, const Params p)
@@ -1096,6 +1113,60 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                 }
             }
             if (threadIdx.x == 0) DSPARK_TRACE_AT(k, 6);
+        }
+
+        if constexpr (kTail) {
+            // ---- the scheduler and the verification, once every score of the launch is
+            // written: ranks by all CTAs (one warp per score), then the last CTA to finish
+            // its ranks scans, picks N*, writes the lengths and verifies every request, with
+            // the same device code as the scheduler and verify kernels
+            __shared__ sched::ScanSmem<kEpiWarps> tail_sm;
+            __shared__ int tail_last;
+            const int n = p.B * p.gamma;
+            if (threadIdx.x == 0) {
+                ctl.go = (ok && wait_counter(p.conf_done, static_cast<uint32_t>(G), p)) ? 1 : 0;
+                DSPARK_TRACE_AT(p.gamma, 22);
+            }
+            epi_sync();
+            const bool go = *reinterpret_cast<volatile int *>(&ctl.go) != 0;
+            // the scores into this CTA's shared memory (the rings are idle once the last
+            // position is drafted: every copy has landed and every MMA has completed), so
+            // that the binary searches read shared memory
+            float *sP = reinterpret_cast<float *>(dyn_smem + (base - smem_u32(dyn_smem)));
+            if (go) {
+#pragma unroll 8
+                for (int i = threadIdx.x; i < n; i += kEpiWarps * 32) sP[i] = __ldcg(p.P_out + i);
+            }
+            epi_sync();
+            if (go)
+                for (int i = blockIdx.x * kEpiWarps + warp; i < n; i += G * kEpiWarps)
+                    sched::rank_score(sP, p.B, p.gamma, n, i, p.rank, sched::LoadPlain{});
+            epi_sync();
+            if (threadIdx.x == 0) DSPARK_TRACE_AT(p.gamma, 23);
+            if (threadIdx.x == 0) {
+                __threadfence();
+                const bool last = atomicAdd(p.tail_done, 1u) == static_cast<unsigned int>(G) - 1u;
+                tail_last = (last && go && !*reinterpret_cast<volatile unsigned int *>(p.abort_flag)) ? 1 : 0;
+                DSPARK_TRACE_AT(p.gamma, 24);
+            }
+            epi_sync();
+            if (tail_last) {
+                __threadfence();
+                // the sorted scores and a copy of the ranks in shared memory, after sP
+                long long *sQ = reinterpret_cast<long long *>(sP + ((n + 1) & ~1));
+                int32_t *sRank = reinterpret_cast<int32_t *>(sQ + n);
+                sched::scan_and_lengths<kEpiWarps>(p.P_out, p.B, p.gamma, n, p.Tstep, p.rank, sQ,
+                                                   p.L_out, p.N_out, p.objective_out, tail_sm,
+                                                   static_cast<int>(threadIdx.x),
+                                                   [] { epi_sync(); }, sRank);
+                epi_sync();
+                if (threadIdx.x == 0) DSPARK_TRACE_AT(p.gamma, 25);
+                for (int b = threadIdx.x; b < p.B; b += kEpiWarps * 32)
+                    verify::verify_request(p.x_out, p.L_out, p.target, b, p.gamma, p.accepted_out,
+                                           p.bonus_out);
+                epi_sync();
+                if (threadIdx.x == 0) DSPARK_TRACE_AT(p.gamma, 26);
+            }
         }
     }
 

@@ -41,15 +41,25 @@ struct Params {
 // to +0.0 as a number) is mapped onto +0.0 by adding +0.0.
 __device__ __forceinline__ uint32_t score_bits(float p) { return __float_as_uint(p + 0.0f); }
 
+// How phase 1 reads the scores: through the read-only path when they are an input of
+// the launch, or with plain loads (a copy in shared memory, say).
+struct LoadReadOnly {
+    __device__ __forceinline__ float operator()(const float *p) const { return __ldg(p); }
+};
+struct LoadPlain {
+    __device__ __forceinline__ float operator()(const float *p) const { return *p; }
+};
+
 // Number of entries of row `row` ordered before the score (bits pb, flat index ib).
+template <typename Load>
 __device__ __forceinline__ int count_before(const float *__restrict__ P, int gamma, int row,
-                                            uint32_t pb, int ib)
+                                            uint32_t pb, int ib, Load ld)
 {
     const float *pr = P + static_cast<size_t>(row) * gamma;
     int lo = 0, hi = gamma;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        const uint32_t m = score_bits(__ldg(pr + mid));
+        const uint32_t m = score_bits(ld(pr + mid));
         const bool before = (m > pb) || (m == pb && row * gamma + mid < ib);
         if (before)
             lo = mid + 1;
@@ -59,96 +69,118 @@ __device__ __forceinline__ int count_before(const float *__restrict__ P, int gam
     return lo;
 }
 
-__device__ __forceinline__ long long block_exclusive_scan(long long v, long long *s_warp,
-                                                          long long &total)
+// Phase 1 for score i, by one warp: its rank (the sum over rows of a binary search),
+// written to rank[i]; a score outside [0, 1] or above its predecessor records
+// DSPARK_NOT_MONOTONE.
+template <typename Load>
+__device__ __forceinline__ void rank_score(const float *__restrict__ P, int B, int gamma, int n,
+                                           int i, int32_t *rank, Load ld)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31;
+    const float pi = ld(P + i);
+    const uint32_t pb = score_bits(pi);
+    int cnt = 0;
+    for (int row = lane; row < B; row += 32) cnt += count_before(P, gamma, row, pb, i, ld);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, o);
+    if (lane == 0) {
+        const int k = i % gamma;
+        const bool bad = !(pi >= 0.0f && pi <= 1.0f) || (k > 0 && pi > ld(P + i - 1));
+        if (bad) record_error(DSPARK_NOT_MONOTONE);
+        rank[i] = min(max(cnt, 0), n - 1);
+    }
+}
+
+// Shared scratch of phase 2 for a group of kW warps.
+template <int kW>
+struct ScanSmem {
+    long long warp_sum[kW];
+    double best_F[kW];
+    int best_N[kW];
+};
+
+// Exclusive scan of one int64 per thread over the group's kW warps (threads t = 0 ..
+// 32 kW - 1 of the group, which `sync` synchronises); `total` gets the sum.
+template <int kW, typename Sync>
+__device__ __forceinline__ long long group_exclusive_scan(long long v, ScanSmem<kW> &sm, int t,
+                                                          Sync sync, long long &total)
+{
+    const int warp = t >> 5, lane = t & 31;
     long long incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const long long t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += t;
+        const long long u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += u;
     }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
+    if (lane == 31) sm.warp_sum[warp] = incl;
+    sync();
     if (warp == 0) {
-        long long w = (lane < kWarps) ? s_warp[lane] : 0;
+        long long w = (lane < kW) ? sm.warp_sum[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const long long t = __shfl_up_sync(0xFFFFFFFFu, w, o);
-            if (lane >= o) w += t;
+            const long long u = __shfl_up_sync(0xFFFFFFFFu, w, o);
+            if (lane >= o) w += u;
         }
-        if (lane < kWarps) s_warp[lane] = w;   // inclusive warp prefix
+        if (lane < kW) sm.warp_sum[lane] = w;   // inclusive warp prefix
     }
-    __syncthreads();
-    total = s_warp[kWarps - 1];
-    const long long before_warp = (warp == 0) ? 0 : s_warp[warp - 1];
+    sync();
+    total = sm.warp_sum[kW - 1];
+    const long long before_warp = (warp == 0) ? 0 : sm.warp_sum[warp - 1];
+    sync();                                     // warp_sum is free again when this returns
     return before_warp + incl - v;
 }
 
-__global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params p)
+// Phase 2, by one group of kW warps (thread t of 32 kW) once every rank is written (ranks
+// and scores are read through L2: other CTAs wrote them): scatter the fixed-point scores
+// q = floor(P 2^46) into rank order, prefix-sum them in int64, evaluate
+// F(N) = double(B 2^46 + S_N) / Tstep[B + N] for every N, take the first maximum (largest
+// F, then smallest N), and count each request's entries ranked below it.  q_sorted is
+// this group's own scratch (global or shared memory); s_rank, when not null, is shared
+// memory for a copy of the ranks, so that the counts read shared memory.
+template <int kW, typename Sync>
+__device__ void scan_and_lengths(const float *__restrict__ P, int B, int gamma, int n,
+                                 const double *__restrict__ Tstep, const int32_t *rank,
+                                 long long *q_sorted, int32_t *L_out, int32_t *N_out,
+                                 double *objective_out, ScanSmem<kW> &sm, int t, Sync sync,
+                                 int32_t *s_rank = nullptr)
 {
-    __shared__ long long s_warp[kWarps];
-    __shared__ double s_bestF[kWarps];
-    __shared__ int s_bestN[kWarps];
-    __shared__ int s_last;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // ---------------- phase 1: ranks
-    for (int i = blockIdx.x * kWarps + warp; i < p.n; i += gridDim.x * kWarps) {
-        const float pi = __ldg(p.P + i);
-        const uint32_t pb = score_bits(pi);
-        int cnt = 0;
-        for (int row = lane; row < p.B; row += 32) cnt += count_before(p.P, p.gamma, row, pb, i);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, o);
-        if (lane == 0) {
-            const int k = i % p.gamma;
-            const bool bad = !(pi >= 0.0f && pi <= 1.0f) || (k > 0 && pi > __ldg(p.P + i - 1));
-            if (bad) record_error(DSPARK_NOT_MONOTONE);
-            p.rank[i] = min(max(cnt, 0), p.n - 1);
-        }
+    constexpr int kT = 32 * kW;
+    const int warp = t >> 5, lane = t & 31;
+    // the loops below are unrolled so that their independent loads are in flight together
+#pragma unroll 8
+    for (int i = t; i < n; i += kT) {
+        const int pos = __ldcg(rank + i);
+        const float pi = __ldcg(P + i);
+        q_sorted[pos] = __float2ll_rz(pi * 0x1p46f);
+        if (s_rank) s_rank[i] = pos;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        s_last = (atomicAdd(p.done, 1u) == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+    sync();
 
-    // ---------------- phase 2 (last CTA): scatter, scan, objective, lengths
-    for (int i = threadIdx.x; i < p.n; i += kThreads) {
-        const int pos = __ldcg(p.rank + i);
-        const float pi = __ldg(p.P + i);
-        p.q_sorted[pos] = __float2ll_rz(pi * 0x1p46f);
-    }
-    __syncthreads();
-
-    const int per = (p.n + kThreads - 1) / kThreads;
-    const int lo = min(p.n, static_cast<int>(threadIdx.x) * per);
-    const int hi = min(p.n, lo + per);
+    const int per = (n + kT - 1) / kT;
+    const int lo = min(n, t * per);
+    const int hi = min(n, lo + per);
     long long part = 0;
-    for (int i = lo; i < hi; ++i) part += __ldcg(p.q_sorted + i);
+#pragma unroll 8
+    for (int i = lo; i < hi; ++i) part += q_sorted[i];
     long long total;
-    long long S = block_exclusive_scan(part, s_warp, total);
+    long long S = group_exclusive_scan<kW>(part, sm, t, sync, total);
 
-    const long long base = static_cast<long long>(p.B) << 46;
+    const long long base = static_cast<long long>(B) << 46;
     double best = -1.0;
     int bestN = 0;
-    if (threadIdx.x == 0) {
-        const double t = __ldg(p.Tstep + p.B);
-        if (!(t > 0.0)) record_error(DSPARK_INVALID_ARG);
-        best = __ll2double_rn(base) / t;
+    if (t == 0) {
+        const double tb = __ldg(Tstep + B);
+        if (!(tb > 0.0)) record_error(DSPARK_INVALID_ARG);
+        best = __ll2double_rn(base) / tb;
         bestN = 0;
     }
+#pragma unroll 8
     for (int i = lo; i < hi; ++i) {
-        S += __ldcg(p.q_sorted + i);
+        S += q_sorted[i];
         const int N = i + 1;
-        const double t = __ldg(p.Tstep + p.B + N);
-        if (!(t > 0.0)) record_error(DSPARK_INVALID_ARG);
-        const double F = __ll2double_rn(base + S) / t;
+        const double tN = __ldg(Tstep + B + N);
+        if (!(tN > 0.0)) record_error(DSPARK_INVALID_ARG);
+        const double F = __ll2double_rn(base + S) / tN;
         if (F > best) {
             best = F;
             bestN = N;
@@ -165,29 +197,58 @@ __global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params 
         }
     }
     if (lane == 0) {
-        s_bestF[warp] = best;
-        s_bestN[warp] = bestN;
+        sm.best_F[warp] = best;
+        sm.best_N[warp] = bestN;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < kWarps; ++w) {
-            if (s_bestF[w] > s_bestF[0] || (s_bestF[w] == s_bestF[0] && s_bestN[w] < s_bestN[0])) {
-                s_bestF[0] = s_bestF[w];
-                s_bestN[0] = s_bestN[w];
+    sync();
+    if (t == 0) {
+        for (int w = 1; w < kW; ++w) {
+            if (sm.best_F[w] > sm.best_F[0] || (sm.best_F[w] == sm.best_F[0] && sm.best_N[w] < sm.best_N[0])) {
+                sm.best_F[0] = sm.best_F[w];
+                sm.best_N[0] = sm.best_N[w];
             }
         }
-        *p.N_out = s_bestN[0];
-        *p.objective_out = s_bestF[0] * 0x1p-46;
-        *p.done = 0u;
+        *N_out = sm.best_N[0];
+        *objective_out = sm.best_F[0] * 0x1p-46;
+    }
+    sync();
+    const int Nstar = sm.best_N[0];
+    // L_b: one warp per request, a ballot over its gamma <= 64 ranks
+    for (int b = warp; b < B; b += kW) {
+        const int32_t *rb = s_rank ? s_rank + b * gamma : rank + b * gamma;
+        int L = 0;
+        for (int k0 = 0; k0 < gamma; k0 += 32) {
+            const int k = k0 + lane;
+            const bool below = k < gamma && (s_rank ? rb[k] : __ldcg(rb + k)) < Nstar;
+            L += __popc(__ballot_sync(0xFFFFFFFFu, below));
+        }
+        if (lane == 0) L_out[b] = L;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) schedule_prefix_kernel(const Params p)
+{
+    __shared__ ScanSmem<kWarps> sm;
+    __shared__ int s_last;
+    const int warp = threadIdx.x >> 5;
+
+    // ---------------- phase 1: ranks
+    for (int i = blockIdx.x * kWarps + warp; i < p.n; i += gridDim.x * kWarps)
+        rank_score(p.P, p.B, p.gamma, p.n, i, p.rank, LoadReadOnly{});
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = (atomicAdd(p.done, 1u) == gridDim.x - 1);
     }
     __syncthreads();
-    const int Nstar = s_bestN[0];
-    for (int b = threadIdx.x; b < p.B; b += kThreads) {
-        int L = 0;
-        for (int k = 0; k < p.gamma; ++k)
-            L += (__ldcg(p.rank + b * p.gamma + k) < Nstar) ? 1 : 0;
-        p.L_out[b] = L;
-    }
+    if (!s_last) return;
+    __threadfence();
+
+    // ---------------- phase 2 (last CTA): scatter, scan, objective, lengths
+    scan_and_lengths<kWarps>(p.P, p.B, p.gamma, p.n, p.Tstep, p.rank, p.q_sorted, p.L_out,
+                             p.N_out, p.objective_out, sm, static_cast<int>(threadIdx.x),
+                             [] { __syncthreads(); });
+    if (threadIdx.x == 0) *p.done = 0u;
 }
 
 }  // namespace sched

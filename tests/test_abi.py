@@ -88,6 +88,30 @@ def test_draft_confidence_step_host_checks():
     assert call(wsb=100) == 3
 
 
+def test_step_host_checks():
+    lib = ds.load()
+    f = lib.dspark_step
+    args = dict(U=_FAKE, anchor=_FAKE, W1=_FAKE, W2=_FAKE, h=_FAKE, w=_FAKE, b_conf=1.0, T=_FAKE,
+                Tstep=_FAKE, target=_FAKE, B=64, gamma=16, V=151936, r=256, d=4096, mode=0,
+                temperature=1.0, seed=0, b_offset=0, x=_FAKE, lx=_FAKE, c=_FAKE, P=_FAKE,
+                L=_FAKE, N=_FAKE, obj=_FAKE, acc=_FAKE, bonus=_FAKE, ws=_FAKE, wsb=1 << 30,
+                stream=None)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return f(a["U"], a["anchor"], a["W1"], a["W2"], a["h"], a["w"], a["b_conf"], a["T"],
+                 a["Tstep"], a["target"], a["B"], a["gamma"], a["V"], a["r"], a["d"], a["mode"],
+                 a["temperature"], a["seed"], a["b_offset"], a["x"], a["lx"], a["c"], a["P"],
+                 a["L"], a["N"], a["obj"], a["acc"], a["bonus"], a["ws"], a["wsb"], a["stream"])
+
+    assert call(Tstep=None) == 1 and call(bonus=None) == 1 and call(target=None) == 1
+    assert call(obj=C.c_void_p(0x10004)) == 1          # fp64 output not 8-byte aligned
+    assert call(B=1024, gamma=65) == 2                  # B gamma above the scheduler's limit
+    assert call(wsb=100) == 3
+    assert call(h=None) == 1 and call(d=1020) == 2      # the confidence checks apply (B <= 128)
+    assert call(U=None) == 1                            # and the drafting checks
+
+
 def test_schedule_and_verify_host_checks():
     lib = ds.load()
     s = lib.dspark_schedule_prefix
