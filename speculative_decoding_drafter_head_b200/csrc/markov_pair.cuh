@@ -52,10 +52,12 @@ constexpr int kW2StageBytes = 64 * kKSlice * 2;       // 64 columns x 128 K rows
 constexpr int kUSlots = 6;
 constexpr int kUSlotBytes = kRows * kUBoxCols * 2;    // 128 rows x 64 columns: 16 KB
 constexpr int kDynSmem = kW2Stages * kW2StageBytes + kUSlots * kUSlotBytes + 1024;
-// TMEM (512 columns): three 128-column accumulators, then A = W1[x_{k-1}] of the CTA's
-// 128 rows (row m in lane m, K = 256 bf16 packed two per column: 128 columns)
-constexpr int kPairAcc = 3;
-constexpr uint32_t kACol = kPairAcc * kAccCols;       // 384
+// TMEM (512 columns): two 128-column accumulators, then two buffers of A = W1[x_{k-1}]
+// for the CTA's 128 rows (row m in lane m, K = 256 bf16 packed two per column: 128
+// columns each), so that the next pass's rows are in place before its first MMA
+constexpr int kPairAcc = 2;
+constexpr int kABufs = 2;
+constexpr uint32_t kACol = kPairAcc * kAccCols;       // 256: A buffer b at 256 + 128 b
 constexpr int kMaxPasses = kMaxB / kPairRows;         // 256-request blocks: 4
 constexpr int kChunks = 4;                            // 32-column chunks of a tile
 constexpr int kBoxWarps = 2 * 4;                      // warps reading one U box: 2 chunks x 4 quadrants
@@ -70,8 +72,8 @@ struct Ctl {
     unsigned long long u_empty[kUSlots];
     unsigned long long tfull[kPairAcc];      // both: the accumulator holds a tile
     unsigned long long tempty[kPairAcc];     // even CTA: all 32 epilogue warps have read it
-    unsigned long long afull;                // even CTA: all 32 epilogue warps gathered A
-    unsigned long long aempty;               // both: the pair MMAs no longer read A
+    unsigned long long afull[kABufs];        // even CTA: all 32 epilogue warps gathered A
+    unsigned long long aempty[kABufs];       // both: the pair MMAs no longer read A
     unsigned long long drain;
     uint32_t tmem_base;
     int abort;
@@ -309,8 +311,8 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
     const uint32_t bar_u_empty = smem_u32(&ctl.u_empty[0]);
     const uint32_t bar_tfull = smem_u32(&ctl.tfull[0]);
     const uint32_t bar_tempty = smem_u32(&ctl.tempty[0]);
-    const uint32_t bar_afull = smem_u32(&ctl.afull);
-    const uint32_t bar_aempty = smem_u32(&ctl.aempty);
+    const uint32_t bar_afull = smem_u32(&ctl.afull[0]);
+    const uint32_t bar_aempty = smem_u32(&ctl.aempty[0]);
     const uint32_t bar_drain = smem_u32(&ctl.drain);
 
     if (threadIdx.x == 0) {
@@ -326,8 +328,10 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
             mbar_init(bar_tfull + 8 * a, 1);
             mbar_init(bar_tempty + 8 * a, 2 * kEpiWarps);
         }
-        mbar_init(bar_afull, 2 * kEpiWarps);
-        mbar_init(bar_aempty, 1);
+        for (int b = 0; b < kABufs; ++b) {
+            mbar_init(bar_afull + 8 * b, 2 * kEpiWarps);
+            mbar_init(bar_aempty + 8 * b, 1);
+        }
         mbar_init(bar_drain, 1);
         ctl.abort = 0;
         mbar_fence_init();
@@ -447,13 +451,14 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
             Ring w2, acc;
             const uint64_t b_desc0 = smem_desc(sW2, kW2StageBytes, 1024, kSwizzle128B);
             const uint16_t both = 0x3;
-            uint32_t a_count = 0;
             bool issued_any = false;
             bool ok = true;
             for (int k = 1; k <= p.gamma && ok; ++k)
                 for (int ps = 0; ps < npass && ok; ++ps) {
                     const int pass = (k - 1) * npass + ps;
-                    if (!wait_bar(bar_afull, a_count & 1u, ctl, p)) {
+                    const int abuf = pass & 1;                    // A buffer of this pass
+                    const uint32_t a_col = kACol + static_cast<uint32_t>(abuf * kAccCols);
+                    if (!wait_bar(bar_afull + 8 * abuf, static_cast<uint32_t>(pass >> 1) & 1u, ctl, p)) {
                         ok = false;
                         break;
                     }
@@ -491,7 +496,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                             for (int kk = 0; kk < kKSlice / 16; ++kk) {
                                 // K elements ks*128 + 16 kk .. + 15: 8 TMEM columns of A
                                 const uint32_t a_tmem =
-                                    tmem + kACol + static_cast<uint32_t>((ks * kKSlice + 16 * kk) >> 1);
+                                    tmem + a_col + static_cast<uint32_t>((ks * kKSlice + 16 * kk) >> 1);
                                 const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
                                 umma_bf16_pair_ts(d_tmem, a_tmem, b_desc, idesc, (ks | kk) ? 1u : 0u);
                             }
@@ -506,8 +511,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                         acc.next(kPairAcc);
                     }
                     if (!ok) break;
-                    umma_commit_pair_mask(bar_aempty, both);
-                    ++a_count;
+                    umma_commit_pair_mask(bar_aempty + 8 * abuf, both);
                 }
             if (issued_any) {
                 umma_commit_pair(bar_drain);
@@ -528,7 +532,6 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
         const uint32_t tempty_lead = mapa_shared(bar_tempty, 0);
         const float c2 = p.inv_tau * kLog2e;
         Ring acc, ur;
-        uint32_t a_count = 0;
         bool ok = true;                                   // uniform within a warp
 
         for (int i = et; i < kMaxPasses * kRows; i += kEpiThreads) {
@@ -538,10 +541,24 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
         }
         epi_sync512();
 
-        // this warp's share of A for pass ps: K elements 64c .. 64c + 63 of the W1 rows of
-        // its quadrant's 32 requests (zeros for rows without a request), loaded into
-        // registers (a whole 128-byte line per lane) and stored into the A columns of TMEM
-        auto gather = [&](int ps) {
+        // this warp's share of A for pass ps of position k (launch-wide pass number P):
+        // K elements 64c .. 64c + 63 of the W1 rows of its quadrant's 32 requests (zeros for
+        // rows without a request), loaded into registers (a whole 128-byte line per lane)
+        // and stored into A buffer P mod 2 of TMEM, once the MMAs of pass P - 2 have
+        // released that buffer.  `wait` false only tests the release; the result says
+        // whether the rows were stored (false also after a failure).
+        auto gather = [&](int k, int ps, bool wait) -> bool {
+            const int P = (k - 1) * npass + ps;
+            const int abuf = P & 1;
+            const uint32_t free_parity = (static_cast<uint32_t>(P >> 1) & 1u) ^ 1u;
+            if (wait) {
+                if (!__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty + 8 * abuf, free_parity, ctl, p))) {
+                    ok = false;
+                    return false;
+                }
+            } else if (!__all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty + 8 * abuf, free_parity))) {
+                return false;
+            }
             const int tok = sh.tok[ps][row];
             uint32_t v[32];
             if (tok >= 0) {
@@ -559,15 +576,15 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0u;
             }
-            tmem_st_32x32b_x32(t_lane + kACol + static_cast<uint32_t>(c * 32), v);
+            tmem_st_32x32b_x32(t_lane + kACol + static_cast<uint32_t>(abuf * kAccCols + c * 32), v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                if (lead) mbar_arrive(bar_afull);
-                else mbar_arrive_remote(afull_lead);
+                if (lead) mbar_arrive(bar_afull + 8 * abuf);
+                else mbar_arrive_remote(afull_lead + 8 * abuf);
             }
-            ++a_count;
+            return true;
         };
 
         // bounded grid barrier number nth; the verdict is taken by one thread and shared, so
@@ -608,10 +625,8 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                     const int tok = sh.tok[ps][row];
                     if (tok >= 0) prefetch_l2(p.W1 + static_cast<size_t>(tok) * kRank + c * 64);
                 }
-                if (__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty, (a_count & 1u) ^ 1u, ctl, p)))
-                    gather(0);
-                else
-                    ok = false;
+                // the rows of the first two passes, each into its own A buffer
+                if (gather(k, 0, true) && npass > 1) gather(k, 1, true);
             }
             for (int ps = 0; ps < npass; ++ps) {
                 const int pass = (k - 1) * npass + ps;
@@ -621,7 +636,9 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                                                         static_cast<uint32_t>(b_row + p.b_offset),
                                                         p.seed_lo, p.seed_hi)
                                             : RowNoise{0u, 0u, 0u, 0u};
-                bool next_gathered = ps + 1 >= npass;
+                // the pass after next reuses this pass's A buffer: its rows go in as soon
+                // as this pass's MMAs are done with it
+                bool next_gathered = ps + 2 >= npass;
                 RowBest best;
                 for (int j = 0; j < ntiles; ++j) {
                     int first, count;
@@ -672,18 +689,9 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                     for (int i = 0; i < nbox; ++i) ur.next(kUSlots);
                     acc.next(kPairAcc);
                     // the next pass's rows are gathered as soon as the MMAs have released A
-                    if (ok && !next_gathered &&
-                        __all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty, (a_count & 1u) ^ 1u))) {
-                        gather(ps + 1);
-                        next_gathered = true;
-                    }
+                    if (ok && !next_gathered && gather(k, ps + 2, false)) next_gathered = true;
                 }
-                if (ok && !next_gathered) {
-                    if (__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty, (a_count & 1u) ^ 1u, ctl, p)))
-                        gather(ps + 1);
-                    else
-                        ok = false;
-                }
+                if (ok && !next_gathered) gather(k, ps + 2, true);
                 // combine the four chunk warps of each row, one atomic per row and CTA
                 sh.part_key[c][row] = argmax_key(best.s, best.v);
                 sh.part_logit[c][row] = best.l;
@@ -728,7 +736,13 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
             epi_sync512();
         }
         // the last pair commit on aempty may still be arriving on this CTA's barrier
-        if (ok) wait_drain(bar_aempty, (a_count & 1u) ^ 1u, p);
+        if (ok) {
+            const int passes = p.gamma * npass;
+            for (int b = 0; b < kABufs; ++b) {
+                const int uses = (passes + 1 - b) / 2;     // passes P < passes with P mod 2 = b
+                if (uses > 0) wait_drain(bar_aempty + 8 * b, static_cast<uint32_t>(uses - 1) & 1u, p);
+            }
+        }
     }
 
     __syncwarp();
