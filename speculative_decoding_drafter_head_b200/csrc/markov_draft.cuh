@@ -29,7 +29,10 @@
 //
 // Warp roles (352 threads): warps 0-7 epilogue and A gather (warps q and q + 4 read
 // TMEM lane quadrant q and take alternate 64-column boxes of each tile), warp 8 W2
-// producer, warp 9 U producer, warp 10 MMA issuer and TMEM owner.  With B <= 64 the MMA
+// producer, warp 9 U producer, warp 10 MMA issuer and TMEM owner; with the confidence
+// head fused in (kConf, 384 threads) warp 11 computes c and P beside the drafting, and
+// with kTail the epilogue warps run the prefix scheduler and the verification after the
+// last position (the scheduler and verify kernels' device code).  With B <= 64 the MMA
 // uses M = 64 (rows 16q..16q+15 sit in TMEM lanes 32q..32q+15, read with 16x256b loads),
 // else M = 128 (32x32b loads).
 #pragma once

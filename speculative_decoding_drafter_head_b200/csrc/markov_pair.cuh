@@ -11,20 +11,22 @@
 // even CTA issues it, each CTA holds the A rows of its own 128 requests and half of the
 // W2 tile's columns, and each CTA's TMEM receives its 128 rows of the accumulator.  Every
 // W2 byte a CTA loads therefore serves 256 requests instead of 128.  The A rows sit in
-// tensor memory (written there by the epilogue warps with tcgen05.st), so the tensor core
-// reads only W2 from shared memory, whose bandwidth the TMA copies and the epilogue's U
-// reads share.  Each pair owns a
-// contiguous vocabulary slice cut into 128-column tiles; for every position k and every
-// block of 256 requests it walks the tiles, alternating direction from one pass to the
-// next, so that the tiles read last are read again first and are still in L2.
+// tensor memory, in two buffers (written there by the epilogue warps with tcgen05.st), so
+// that the next block's rows are in place before its first MMA and the tensor core reads
+// only W2 from shared memory, whose bandwidth the TMA copies and the epilogue's U reads
+// share.  Each pair owns a contiguous vocabulary slice cut into 128-column tiles; for
+// every position k and every block of 256 requests (a pass) it walks the tiles,
+// alternating direction from one pass to the next, so that the tiles read last are read
+// again first and are still in L2.
 //
 // Per CTA: 16 epilogue warps (four per TMEM lane quadrant, one 32-column chunk of every
 // tile each), warp 16 the W2 producer (TMA, 64 columns x 128 K rows per stage), warp 17
 // the U producer (TMA, 128 rows x 64 columns per box), warp 18 the MMA issuer in the even
-// CTA, and in the kConf instances warp 19 the confidence head (as in markov_draft_kernel).  Signals that cross the pair: the odd CTA's W2 copies complete on the even CTA's
-// stage barrier (.cta_group::2 copies; the even CTA arms it for both halves), and its A
-// gathers and accumulator releases arrive on the even CTA's barriers; the even CTA's MMA
-// completions arrive on both CTAs' barriers through one pair commit.
+// CTA, and in the kConf instances warp 19 the confidence head (as in
+// markov_draft_kernel).  Signals that cross the pair: the odd CTA's W2 copies complete
+// on the even CTA's stage barrier (.cta_group::2 copies; the even CTA arms it for both
+// halves), and its A gathers and accumulator releases arrive on the even CTA's barriers;
+// the even CTA's MMA completions arrive on both CTAs' barriers through one pair commit.
 //
 // Selection as in markov_draft_kernel: greedy argmax with the smallest index on ties, or
 // Gumbel-max with Philox noise keyed (seed, request, position, vocabulary index).  Here the
