@@ -1158,15 +1158,16 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                 // the sorted scores and a copy of the ranks in shared memory, after sP
                 long long *sQ = reinterpret_cast<long long *>(sP + ((n + 1) & ~1));
                 int32_t *sRank = reinterpret_cast<int32_t *>(sQ + n);
+                int32_t *sL = sRank + n;
                 sched::scan_and_lengths<kEpiWarps>(p.P_out, p.B, p.gamma, n, p.Tstep, p.rank, sQ,
                                                    p.L_out, p.N_out, p.objective_out, tail_sm,
                                                    static_cast<int>(threadIdx.x),
-                                                   [] { epi_sync(); }, sRank);
+                                                   [] { epi_sync(); }, sRank, sL);
                 epi_sync();
                 if (threadIdx.x == 0) DSPARK_TRACE_AT(p.gamma, 25);
                 for (int b = threadIdx.x; b < p.B; b += kEpiWarps * 32)
-                    verify::verify_request(p.x_out, p.L_out, p.target, b, p.gamma, p.accepted_out,
-                                           p.bonus_out);
+                    verify::verify_request_len(p.x_out, sL[b], p.target, b, p.gamma,
+                                               p.accepted_out, p.bonus_out);
                 epi_sync();
                 if (threadIdx.x == 0) DSPARK_TRACE_AT(p.gamma, 26);
             }

@@ -136,13 +136,14 @@ __device__ __forceinline__ long long group_exclusive_scan(long long v, ScanSmem<
 // F(N) = double(B 2^46 + S_N) / Tstep[B + N] for every N, take the first maximum (largest
 // F, then smallest N), and count each request's entries ranked below it.  q_sorted is
 // this group's own scratch (global or shared memory); s_rank, when not null, is shared
-// memory for a copy of the ranks, so that the counts read shared memory.
+// memory for a copy of the ranks, so that the counts read shared memory, and s_L, when
+// not null, receives the lengths as well.
 template <int kW, typename Sync>
 __device__ void scan_and_lengths(const float *__restrict__ P, int B, int gamma, int n,
                                  const double *__restrict__ Tstep, const int32_t *rank,
                                  long long *q_sorted, int32_t *L_out, int32_t *N_out,
                                  double *objective_out, ScanSmem<kW> &sm, int t, Sync sync,
-                                 int32_t *s_rank = nullptr)
+                                 int32_t *s_rank = nullptr, int32_t *s_L = nullptr)
 {
     constexpr int kT = 32 * kW;
     const int warp = t >> 5, lane = t & 31;
@@ -222,7 +223,10 @@ __device__ void scan_and_lengths(const float *__restrict__ P, int B, int gamma, 
             const bool below = k < gamma && (s_rank ? rb[k] : __ldcg(rb + k)) < Nstar;
             L += __popc(__ballot_sync(0xFFFFFFFFu, below));
         }
-        if (lane == 0) L_out[b] = L;
+        if (lane == 0) {
+            L_out[b] = L;
+            if (s_L) s_L[b] = L;
+        }
     }
 }
 
