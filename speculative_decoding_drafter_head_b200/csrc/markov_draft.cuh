@@ -89,6 +89,10 @@ struct Params {
     int units_total;             // ceil(V / 32)
     int M;                       // requests per MMA tile: 64 (B <= 64) or 128
     int w2_stages;               // W2 ring depth
+    int w2_stage_bytes;          // one K half of a tile: tile_units / 2 boxes of 16 KB
+    int tile_units;              // 32-column units per MMA tile (N = 32 tile_units)
+    int acc_cols;                // TMEM columns of one accumulator (32 tile_units)
+    int acc_slots;               // accumulators in TMEM (512 / acc_cols, at most kAcc)
     int ub;                      // rows of the U TMA box: min(B, M)
     int u_slots;                 // U ring depth (boxes of 64 columns)
     int u_slot_bytes;
@@ -145,6 +149,14 @@ struct Ring {
         }
     }
 };
+
+// The t-th tile of a CTA that owns n_units units, in tiles of `units` units: full tiles,
+// then the remainder.
+__device__ __forceinline__ void tile_span_n(int t, int n_units, int units, int &first, int &count)
+{
+    first = t * units;
+    count = min(units, n_units - first);
+}
 
 // The t-th tile of a CTA that owns n_units units: full tiles of kMaxUnits units, then
 // the remainder (an MMA costs the same for any N <= 128, so this minimises the count).
@@ -615,14 +627,14 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
     const uint32_t base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
     const uint32_t sA = base;
     const uint32_t sW2 = base + static_cast<uint32_t>(M * kRank * 2);
-    const uint32_t sU = sW2 + static_cast<uint32_t>(p.w2_stages * kW2StageBytes);
+    const uint32_t sU = sW2 + static_cast<uint32_t>(p.w2_stages * p.w2_stage_bytes);
 
     const int G = gridDim.x;
     const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * p.units_total / G);
     const int u_end =
         static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.units_total / G);
     const int n_units = u_end - u_begin;
-    const int ntiles = (n_units + kMaxUnits - 1) / kMaxUnits;
+    const int ntiles = (n_units + p.tile_units - 1) / p.tile_units;
     const int num_mt = (p.B + M - 1) / M;
 
     const uint32_t bar_w2_full = smem_u32(&ctl.w2_full[0]);
@@ -678,7 +690,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                 for (int mt = 0; mt < num_mt && ok; ++mt) {
                     for (int t = 0; t < ntiles && ok; ++t) {
                         int first, count;
-                        tile_span(t, n_units, ntiles, first, count);
+                        tile_span_n(t, n_units, p.tile_units, first, count);
                         const int v0 = (u_begin + first) * kUnit;
                         const int nbox = (count + 1) >> 1;          // 64-column boxes
                         if (mt == 0 && t == 0) DSPARK_TRACE_AT(k, 7);
@@ -689,7 +701,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                                 break;
                             }
                             const uint32_t bar = bar_w2_full + 8 * w2.slot;
-                            const uint32_t dst = sW2 + w2.slot * kW2StageBytes;
+                            const uint32_t dst = sW2 + w2.slot * p.w2_stage_bytes;
                             mbar_arrive_expect_tx(bar, nbox * kW2BoxBytes);
                             for (int i = 0; i < nbox; ++i)
                                 tma_load_2d(dst + i * kW2BoxBytes, &tm_w2, bar, v0 + 64 * i,
@@ -714,7 +726,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                 for (int mt = 0; mt < num_mt && ok; ++mt) {
                     for (int t = 0; t < ntiles && ok; ++t) {
                         int first, count;
-                        tile_span(t, n_units, ntiles, first, count);
+                        tile_span_n(t, n_units, p.tile_units, first, count);
                         const int v0 = (u_begin + first) * kUnit;
                         for (int u = 0; u < count; u += 2) {
                             if (!wait_phase(bar_u_empty + 8 * ur.slot, ur.phase ^ 1u, ctl, p)) {
@@ -755,7 +767,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                     tc_fence_after();
                     for (int t = 0; t < ntiles && ok; ++t) {
                         int first, count;
-                        tile_span(t, n_units, ntiles, first, count);
+                        tile_span_n(t, n_units, p.tile_units, first, count);
                         const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(M),
                                                               static_cast<uint32_t>(count * kUnit), 1);
 #ifdef DSPARK_TRACE
@@ -767,7 +779,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                         }
                         DSPARK_TRACE_ADD(k, 14, globaltimer_ns() - tw0);
                         tc_fence_after();
-                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
+                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * p.acc_cols);
                         for (int ks = 0; ks < kKSlices; ++ks) {
 #ifdef DSPARK_TRACE
                             const uint64_t tw1 = globaltimer_ns();
@@ -782,7 +794,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                             // descriptors differ only in the start-address field (bits 0..13,
                             // 16-byte units): advance them with plain adds
                             const uint64_t a_k = a_desc0 + static_cast<uint64_t>((2 * ks * a_chunk) >> 4);
-                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((w2.slot * kW2StageBytes) >> 4);
+                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((w2.slot * p.w2_stage_bytes) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < kKSlice / 16; ++kk) {
                                 const uint64_t a_desc =
@@ -799,7 +811,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                         if (mt == 0 && t == 0) DSPARK_TRACE_AT(k, 9);
                         if (mt == num_mt - 1 && t == ntiles - 1) DSPARK_TRACE_AT(k, 10);
                         umma_commit(bar_tfull + 8 * acc.slot);
-                        acc.next(kAcc);
+                        acc.next(p.acc_slots);
                     }
                     if (!ok) break;
                     umma_commit(bar_aempty);
@@ -986,7 +998,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                 RowBest best64[2];
                 for (int t = 0; t < ntiles; ++t) {
                     int first, count;
-                    tile_span(t, n_units, ntiles, first, count);
+                    tile_span_n(t, n_units, p.tile_units, first, count);
                     const int nbox = (count + 1) >> 1;
 #ifdef DSPARK_TRACE
                     const uint64_t tfw0 = globaltimer_ns();
@@ -1004,11 +1016,14 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                         const uint64_t tbusy0 = globaltimer_ns();
 #endif
                         // box i of the tile holds chunks 2i and 2i + 1; this warp takes boxes
-                        // i = half, half + 2, ... and reduces both chunks of a box together
-                        const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * kAccCols);
+                        // i = s, s + 2, ... and reduces both chunks of a box together, where
+                        // s = half, swapped on odd tiles when a tile has an odd number of
+                        // boxes so that the two warps of a quadrant share them evenly
+                        const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc.slot * p.acc_cols);
+                        const int s0 = ((nbox & 1) && (t & 1)) ? (half ^ 1) : half;
                         Ring my = ur;
-                        if (half) my.next(p.u_slots);
-                        for (int i = half; i < nbox; i += 2) {
+                        if (s0) my.next(p.u_slots);
+                        for (int i = s0; i < nbox; i += 2) {
 #ifdef DSPARK_TRACE
                             const uint64_t tw2 = globaltimer_ns();
 #endif
@@ -1048,7 +1063,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConf : kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar_tempty + 8 * acc.slot);
                     }
-                    acc.next(kAcc);
+                    acc.next(p.acc_slots);
                     if (ok && !next_gathered &&
                         __all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty, (mt_count & 1u) ^ 1u))) {
                         gather(mt + 1);
