@@ -82,8 +82,7 @@ unsigned long long current_ctx_id()
 }
 
 constexpr int kMaxDevices = 64;
-constexpr int kTileUnitsM64 = 6;  // 32-column units per tile of the M = 64 instances
-constexpr int kW2StagesM64 = 3;   // W2 ring depth of the M = 64 instances (48 KB stages)
+constexpr int kTileUnits = 6;     // 32-column units per tile of the single-CTA draft kernel
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -359,14 +358,15 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     prm.units_total = (V + D::kUnit - 1) / D::kUnit;
     prm.M = M;
     // shared memory: A (M x 256 bf16), then the W2 ring, then U boxes in what is left
-    // M = 64: 192-column tiles (6 units; two 192-column accumulators), which cut the
-    // tiles per CTA and leave no CTA with one extra tile at the usual vocabulary sizes;
-    // M = 128: 128-column tiles and four accumulators
-    prm.tile_units = M == 64 ? kTileUnitsM64 : D::kMaxUnits;
+    // 192-column tiles (6 units; two 192-column accumulators): fewer tiles per CTA, and
+    // at the usual vocabulary sizes no CTA with one extra tile (its 33rd unit) that every
+    // position's grid barrier would wait for.  W2 stages of three 64-column boxes per K
+    // half; the ring is 3 deep with M = 64 and 2 with M = 128, whose A tile is twice as big
+    prm.tile_units = kTileUnits;
     prm.acc_cols = prm.tile_units * D::kUnit;
-    prm.acc_slots = M == 64 ? 2 : D::kAcc;
+    prm.acc_slots = 2;
     prm.w2_stage_bytes = ((prm.tile_units + 1) / 2) * D::kW2BoxBytes;
-    prm.w2_stages = M == 64 ? kW2StagesM64 : 3;
+    prm.w2_stages = M == 64 ? 3 : 2;
     prm.ub = ub;
     prm.u_slot_bytes = static_cast<int>(round_up(static_cast<size_t>(ub) * D::kUBoxCols * 2, 1024));
     prm.u_slots = (D::kRingSmem - M * D::kRank * 2 - prm.w2_stages * prm.w2_stage_bytes) /
