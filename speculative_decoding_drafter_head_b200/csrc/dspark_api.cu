@@ -82,7 +82,7 @@ unsigned long long current_ctx_id()
 }
 
 constexpr int kMaxDevices = 64;
-constexpr int kTileUnits = 6;     // 32-column units per tile of the single-CTA draft kernel
+constexpr int kTileUnitsWide = 6; // 32-column units per wide tile of the single-CTA draft kernel
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
@@ -356,17 +356,23 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     prm.a_rows = reinterpret_cast<uint16_t *>(ws + draft_keys_end(B, gamma) +
                                               static_cast<size_t>(B) * 256 * 4);
     prm.units_total = (V + D::kUnit - 1) / D::kUnit;
+    const int grid_single = prm.units_total < dev->sms ? prm.units_total : dev->sms;
     prm.M = M;
     // shared memory: A (M x 256 bf16), then the W2 ring, then U boxes in what is left
-    // 192-column tiles (6 units; two 192-column accumulators): fewer tiles per CTA, and
-    // at the usual vocabulary sizes no CTA with one extra tile (its 33rd unit) that every
-    // position's grid barrier would wait for.  W2 stages of three 64-column boxes per K
-    // half; the ring is 3 deep with M = 64 and 2 with M = 128, whose A tile is twice as big
-    prm.tile_units = kTileUnits;
+    // Tile width: 192 columns (6 units; two 192-column accumulators) where that takes
+    // fewer tiles per CTA than 128 columns (4 units; four accumulators), else 128.  At the
+    // 151936-column vocabularies every CTA then has six tiles instead of eight, or nine for
+    // the CTAs with a 33rd unit, which every position's grid barrier waited for.  W2
+    // stages hold tile_units / 2 boxes of 64 columns per K half; the ring is one stage
+    // deeper with M = 64, whose A tile is half as big.
+    const int per_cta = (prm.units_total + grid_single - 1) / grid_single;
+    const bool wide = (per_cta + kTileUnitsWide - 1) / kTileUnitsWide <
+                      (per_cta + D::kMaxUnits - 1) / D::kMaxUnits;
+    prm.tile_units = wide ? kTileUnitsWide : D::kMaxUnits;
     prm.acc_cols = prm.tile_units * D::kUnit;
-    prm.acc_slots = 2;
+    prm.acc_slots = wide ? 2 : D::kAcc;
     prm.w2_stage_bytes = ((prm.tile_units + 1) / 2) * D::kW2BoxBytes;
-    prm.w2_stages = M == 64 ? 3 : 2;
+    prm.w2_stages = (wide ? 2 : 3) + (M == 64 ? 1 : 0);
     prm.ub = ub;
     prm.u_slot_bytes = static_cast<int>(round_up(static_cast<size_t>(ub) * D::kUBoxCols * 2, 1024));
     prm.u_slots = (D::kRingSmem - M * D::kRank * 2 - prm.w2_stages * prm.w2_stage_bytes) /
@@ -414,8 +420,7 @@ int launch_draft(const void *U, const int32_t *anchor, const void *W1, const voi
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     if (!pair) {
-        const int grid = prm.units_total < dev->sms ? prm.units_total : dev->sms;
-        cfg.gridDim = dim3(grid);
+        cfg.gridDim = dim3(grid_single);
         cfg.blockDim = dim3(fused ? D::kThreadsConf : D::kThreads);
         cfg.numAttrs = 1;
         return from_cuda(cudaLaunchKernelEx(&cfg, kern, tm_w2, tm_u, prm));
