@@ -87,32 +87,108 @@ def _traffic_per_launch(workload_name, gamma):
     return None
 
 
+_NVML_SAMPLER = r"""
+import sys, time
+import pynvml as N
+N.nvmlInit()
+uuid, index, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+h = None
+if uuid:
+    try:
+        h = N.nvmlDeviceGetHandleByUUID(uuid)
+    except Exception:
+        h = None
+if h is None:
+    h = N.nvmlDeviceGetHandleByIndex(index)
+mx = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+print("ready", mx, flush=True)
+while True:
+    t = time.monotonic_ns()
+    sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+    why = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+    mw = N.nvmlDeviceGetPowerUsage(h)
+    print(t, sm, why, mw, flush=True)
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and clock-event reasons sampled by NVML in a separate process (every
+    0.5 ms, so the GIL and the host's synchronize do not hold it up) with timestamps on
+    the host's monotonic clock; only the samples taken between begin() and end() -- the
+    timed region -- are summarised.  Falls back to nvidia-smi (200 ms) without NVML."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h): sw power cap 0x4, hw slowdown 0x8,
+    # sw thermal 0x20, hw thermal 0x40, hw power brake 0x80
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8 | 0x80, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
+        self.mode = None
+        self.max_mhz = None
+
+    def _nvml_target(self):
+        """(uuid, NVML index) of the CUDA device this process drives."""
+        uuid = ""
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+            if u:
+                uuid = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:                               # noqa: BLE001
+            pass
+        index = self.index
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v for v in vis.split(",") if v.strip()]
+        if ids and all(v.strip().isdigit() for v in ids) and self.index < len(ids):
+            index = int(ids[self.index])
+        return uuid, index
 
     def start(self):
         try:
+            uuid, index = self._nvml_target()
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                [sys.executable, "-c", _NVML_SAMPLER, uuid, str(index), "0.0005"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except Exception:
+            first = self.proc.stdout.readline().split()
+            if len(first) == 2 and first[0] == "ready":
+                self.mode, self.max_mhz = "nvml", float(first[1])
+            else:
+                self.proc.kill()
+                self.proc = None
+        except Exception:                               # noqa: BLE001
             self.proc = None
+        if self.proc is None:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.mode = "nvidia-smi"
+            except Exception:                           # noqa: BLE001
+                self.proc = None
+                return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic_ns(), line.strip()))
+
+    def begin(self):
+        """Start of the timed region (after the synchronize that opens it)."""
+        self.t0 = time.monotonic_ns()
+
+    def end(self):
+        """End of the timed region (after the synchronize that closes it)."""
+        self.t1 = time.monotonic_ns()
 
     def stop(self):
         if self.proc is None:
@@ -120,27 +196,47 @@ class ClockSampler:
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
-        except Exception:
+        except Exception:                               # noqa: BLE001
             self.proc.kill()
         self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+        t0 = self.t0 if self.t0 is not None else 0
+        t1 = self.t1 if self.t1 is not None else 2 ** 63
+        rows = []                               # (t, sm MHz, max MHz, reasons, watts)
+        if self.mode == "nvml":
+            for _, ln in self.lines:
+                parts = ln.split()
+                if len(parts) != 4:
+                    continue
+                t, sm, why = int(parts[0]), float(parts[1]), int(parts[2])
+                rows.append((t, sm, self.max_mhz,
+                             {n for n, bit in self.BITS.items() if why & bit},
+                             float(parts[3]) / 1e3))
+        else:
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                     "sw_power_cap"]
+            for t, ln in self.lines:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, mx, w = float(parts[1]), float(parts[2]), float(parts[3])
+                except ValueError:
+                    continue
+                rows.append((t, sm, mx, {n for n, v in zip(names, parts[5:9])
+                                         if v.lower().startswith("active")}, w))
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        if not inside:                                  # region shorter than one period:
+            after = [r for r in rows if r[0] >= t0]     # the first sample after it began
+            inside = after[:1]
+        if not inside:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set().union(*(r[3] for r in inside))
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_min_mhz": min(r[1] for r in inside), "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(reasons), "samples": len(inside),
+                "power_w": round(statistics.median(r[4] for r in inside), 1),
+                "source": self.mode,
+                "window_ms": round((t1 - t0) / 1e6, 3) if self.t1 is not None else None}
 
 
 def workload_config(wl, world=1):
@@ -299,7 +395,8 @@ def run_sts_fit(args):
     assert ds.get_error() == 0
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
     clocks.start()
-    time.sleep(0.5)
+    time.sleep(0.05)
+    clocks.begin()
     evs = []
     for _ in range(args.steps):
         e0 = torch.cuda.Event(enable_timing=True)
@@ -309,6 +406,7 @@ def run_sts_fit(args):
         e1.record(stream)
         evs.append((e0, e1))
     torch.cuda.synchronize()
+    clocks.end()
     clk = clocks.stop()
     ms = [a.elapsed_time(b) for a, b in evs]
     evals = float(N) * gamma * n_t
@@ -558,10 +656,11 @@ def main():
 
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.5)
+    time.sleep(0.05)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    clocks.begin()
     step_ev = []
     for _ in range(args.steps):
         flush.zero_()                                   # evict L2 between timed steps
@@ -572,6 +671,7 @@ def main():
         e1.record(stream)
         step_ev.append((e0, e1))
     torch.cuda.synchronize()
+    clocks.end()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()

@@ -54,3 +54,26 @@ def test_parity_report_counts_mismatches(oracle_mod):
     bad["x"][b, k] = (x[b, k] + 1) % wl.V
     rep = bench.parity_report(wl, inp, target, bad, oracle_mod, schedule=False)
     assert not rep["ok"] and rep["hard_mismatch"] >= 1
+
+
+def test_clock_sampler_keeps_the_timed_region():
+    """Only the NVML samples stamped between begin() and end() are summarised, and the
+    clock-event bits map onto the reason names the record uses."""
+    import types
+    import bench
+    s = bench.ClockSampler(0)
+    s.mode, s.max_mhz = "nvml", 1965.0
+    ms = 1_000_000
+    # ten samples 1 ms apart; the one at 3 ms has the sw power cap bit, the one at 8 ms
+    # (outside the region) the hw slowdown bit
+    s.lines = [(0, f"{i * ms} {1965 - 10 * i} {4 if i == 3 else (8 if i == 8 else 0)} "
+                   f"{(600 + i) * 1000}") for i in range(10)]
+    s.t0, s.t1 = 2 * ms, 5 * ms
+    s.proc = types.SimpleNamespace(terminate=lambda: None, wait=lambda timeout=None: None,
+                                   kill=lambda: None)
+    s.thread = types.SimpleNamespace(join=lambda timeout=None: None)
+    clk = s.stop()
+    assert clk["samples"] == 4 and clk["source"] == "nvml"
+    assert clk["sm_mhz"] == 1965 - 35 and clk["sm_min_mhz"] == 1965 - 50
+    assert clk["reasons"] == ["sw_power_cap"] and clk["window_ms"] == 3.0
+    assert clk["power_w"] == 603.5
