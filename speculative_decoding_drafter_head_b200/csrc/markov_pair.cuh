@@ -156,10 +156,19 @@ __device__ __forceinline__ bool drain_or_settle(uint32_t bar0, int n, long long 
     return true;
 }
 
-// The j-th tile of pass `pass`: forward on even passes, backward on odd ones.
-__device__ __forceinline__ int snake(int pass, int j, int ntiles)
+// The j-th tile of super-pass S: forward on even super-passes, backward on odd ones.
+__device__ __forceinline__ int snake(int S, int j, int ntiles)
 {
-    return (pass & 1) ? ntiles - 1 - j : j;
+    return (S & 1) ? ntiles - 1 - j : j;
+}
+
+// Request block ps always reads A buffer ps mod 2.  Uses of that buffer before block ps
+// of position k: every earlier position's blocks of the same parity, and this position's
+// blocks ps - 2, ps - 4, ...
+__device__ __forceinline__ uint32_t abuf_uses(int k, int ps, int npass)
+{
+    const int per_position = (ps & 1) ? npass / 2 : (npass + 1) / 2;
+    return static_cast<uint32_t>((k - 1) * per_position + (ps >> 1));
 }
 
 // ------------------------------------------------------------------ Philox, one request row
@@ -306,6 +315,21 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
     const int n_units = u_end - u_begin;
     const int ntiles = (n_units + kMaxUnits - 1) / kMaxUnits;
     const int npass = (p.B + kPairRows - 1) / kPairRows;   // 256-request blocks per position
+    // super-pass: the request blocks that take their MMAs from the same W2 stages, tile by
+    // tile (two for greedy drafting; one for Gumbel-max, whose selection arithmetic, not
+    // the W2 stream, bounds it)
+    constexpr int kSpMax = kGumbel ? 1 : 2;
+    const int nsp = (npass + kSpMax - 1) / kSpMax;          // super-passes per position
+    auto sp_blocks = [&](int sp) { return min(kSpMax, npass - kSpMax * sp); };
+    // A buffer of block ps at position k, and its uses before that: the block's parity with
+    // two blocks per super-pass; with one, the launch-wide pass number's parity (so that
+    // consecutive passes, also across positions, alternate)
+    auto a_buf = [&](int k, int ps) -> int {
+        return kSpMax == 2 ? (ps & 1) : (((k - 1) * npass + ps) & 1);
+    };
+    auto a_uses = [&](int k, int ps) -> uint32_t {
+        return kSpMax == 2 ? abuf_uses(k, ps, npass) : static_cast<uint32_t>(((k - 1) * npass + ps) >> 1);
+    };
 
     const uint32_t bar_w2_full = smem_u32(&ctl.w2_full[0]);
     const uint32_t bar_w2_empty = smem_u32(&ctl.w2_empty[0]);
@@ -360,11 +384,12 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
             long long issued = 0;
             bool ok = true;
             for (int k = 1; k <= p.gamma && ok; ++k)
-                for (int ps = 0; ps < npass && ok; ++ps) {
-                    const int pass = (k - 1) * npass + ps;
+                for (int sp = 0; sp < nsp && ok; ++sp) {
+                    const int S = (k - 1) * nsp + sp;
+                    [[maybe_unused]] const int ps = kSpMax * sp;
                     for (int j = 0; j < ntiles && ok; ++j) {
                         int first, count;
-                        tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                        tile_span(snake(S, j, ntiles), n_units, ntiles, first, count);
                         // this CTA's half of the tile: columns rank * N/2 .. + N/2 (a 64-column box)
                         const int x = (u_begin + first) * kUnit + static_cast<int>(rank) * count * (kUnit / 2);
                         for (int ks = 0; ks < kKSlices; ++ks) {
@@ -401,25 +426,29 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
             long long issued = 0;
             bool ok = true;
             for (int k = 1; k <= p.gamma && ok; ++k)
-                for (int ps = 0; ps < npass && ok; ++ps) {
-                    const int pass = (k - 1) * npass + ps;
-                    const int row0 = ps * kPairRows + static_cast<int>(rank) * kRows;
+                for (int sp = 0; sp < nsp && ok; ++sp) {
+                    const int S = (k - 1) * nsp + sp;
+                    const int nb = sp_blocks(sp);
                     for (int j = 0; j < ntiles && ok; ++j) {
                         int first, count;
-                        tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                        tile_span(snake(S, j, ntiles), n_units, ntiles, first, count);
                         const int v0 = (u_begin + first) * kUnit;
-                        for (int u = 0; u < count; u += 2) {
-                            if (!wait_bar(bar_u_empty + 8 * ur.slot, ur.phase ^ 1u, ctl, p)) {
-                                ok = false;
-                                break;
+                        for (int bi = 0; bi < nb && ok; ++bi) {
+                            const int ps = kSpMax * sp + bi;
+                            const int row0 = ps * kPairRows + static_cast<int>(rank) * kRows;
+                            for (int u = 0; u < count; u += 2) {
+                                if (!wait_bar(bar_u_empty + 8 * ur.slot, ur.phase ^ 1u, ctl, p)) {
+                                    ok = false;
+                                    break;
+                                }
+                                PAIR_TRACE(k, ps, j, 10 + u / 2);
+                                const uint32_t bar = bar_u_full + 8 * ur.slot;
+                                mbar_arrive_expect_tx(bar, kUSlotBytes);
+                                tma_load_3d(sU + ur.slot * kUSlotBytes, &tm_u, bar, v0 + u * kUnit, k - 1,
+                                            row0, pol_u);
+                                ++issued;
+                                ur.next(kUSlots);
                             }
-                            PAIR_TRACE(k, ps, j, 10 + u / 2);
-                            const uint32_t bar = bar_u_full + 8 * ur.slot;
-                            mbar_arrive_expect_tx(bar, kUSlotBytes);
-                            tma_load_3d(sU + ur.slot * kUSlotBytes, &tm_u, bar, v0 + u * kUnit, k - 1,
-                                        row0, pol_u);
-                            ++issued;
-                            ur.next(kUSlots);
                         }
                     }
                 }
@@ -456,64 +485,75 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
             bool issued_any = false;
             bool ok = true;
             for (int k = 1; k <= p.gamma && ok; ++k)
-                for (int ps = 0; ps < npass && ok; ++ps) {
-                    const int pass = (k - 1) * npass + ps;
-                    const int abuf = pass & 1;                    // A buffer of this pass
-                    const uint32_t a_col = kACol + static_cast<uint32_t>(abuf * kAccCols);
-                    if (!wait_bar(bar_afull + 8 * abuf, static_cast<uint32_t>(pass >> 1) & 1u, ctl, p)) {
-                        ok = false;
-                        break;
+                for (int sp = 0; sp < nsp && ok; ++sp) {
+                    const int S = (k - 1) * nsp + sp;
+                    const int nb = sp_blocks(sp);
+                    // block ps = kSpMax sp + bi reads A buffer ps mod 2
+                    for (int bi = 0; bi < nb && ok; ++bi) {
+                        const int ps = kSpMax * sp + bi;
+                        if (!wait_bar(bar_afull + 8 * a_buf(k, ps), a_uses(k, ps) & 1u, ctl, p))
+                            ok = false;
                     }
+                    if (!ok) break;
                     tc_fence_after();
                     for (int j = 0; j < ntiles && ok; ++j) {
+                        [[maybe_unused]] const int ps = kSpMax * sp;
                         int first, count;
-                        tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                        tile_span(snake(S, j, ntiles), n_units, ntiles, first, count);
                         const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(kPairRows),
                                                               static_cast<uint32_t>(count * kUnit), 1);
-                        PAIR_TRACE(k, ps, j, 0);
-                        if (!wait_bar(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p)) {
-                            ok = false;
-                            break;
-                        }
-                        PAIR_TRACE(k, ps, j, 1);
                         static_assert(kKSlices == 2, "a tile's K is two W2 stages");
-                        // both K halves are waited for up front, so that the tile's 16 MMAs
-                        // issue back to back: the tensor core's queue is short, and a wait
-                        // between them leaves it idle
+                        // both K halves are waited for up front, so that the tile's MMAs issue
+                        // back to back: the tensor core's queue is short, and a wait between
+                        // them leaves it idle.  Every block of the super-pass then takes its 16
+                        // MMAs from the same two stages, into its own accumulator.
                         Ring w2b = w2;
                         w2b.next(kW2Stages);
-                        if (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p) ||
-                            !wait_bar(bar_w2_full + 8 * w2b.slot, w2b.phase, ctl, p)) {
-                            ok = false;
-                            break;
-                        }
-                        PAIR_TRACE(k, ps, j, 2);
-                        tc_fence_after();
-                        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
 #pragma unroll
-                        for (int ks = 0; ks < kKSlices; ++ks) {
-                            const uint32_t slot = ks ? w2b.slot : w2.slot;
-                            const uint64_t b_k = b_desc0 + static_cast<uint64_t>((slot * kW2StageBytes) >> 4);
-#pragma unroll
-                            for (int kk = 0; kk < kKSlice / 16; ++kk) {
-                                // K elements ks*128 + 16 kk .. + 15: 8 TMEM columns of A
-                                const uint32_t a_tmem =
-                                    tmem + a_col + static_cast<uint32_t>((ks * kKSlice + 16 * kk) >> 1);
-                                const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
-                                umma_bf16_pair_ts(d_tmem, a_tmem, b_desc, idesc, (ks | kk) ? 1u : 0u);
+                        for (int bi = 0; bi < kSpMax; ++bi) {
+                            if (bi >= nb) break;
+                            PAIR_TRACE(k, ps + bi, j, 0);
+                            if (!wait_bar(bar_tempty + 8 * acc.slot, acc.phase ^ 1u, ctl, p)) {
+                                ok = false;
+                                break;
                             }
+                            PAIR_TRACE(k, ps + bi, j, 1);
+                            if (bi == 0 && (!wait_bar(bar_w2_full + 8 * w2.slot, w2.phase, ctl, p) ||
+                                            !wait_bar(bar_w2_full + 8 * w2b.slot, w2b.phase, ctl, p))) {
+                                ok = false;
+                                break;
+                            }
+                            PAIR_TRACE(k, ps + bi, j, 2);
+                            tc_fence_after();
+                            const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
+                            const uint32_t a_col = kACol + static_cast<uint32_t>(a_buf(k, ps + bi) * kAccCols);
+#pragma unroll
+                            for (int ks = 0; ks < kKSlices; ++ks) {
+                                const uint32_t slot = ks ? w2b.slot : w2.slot;
+                                const uint64_t b_k = b_desc0 + static_cast<uint64_t>((slot * kW2StageBytes) >> 4);
+#pragma unroll
+                                for (int kk = 0; kk < kKSlice / 16; ++kk) {
+                                    // K elements ks*128 + 16 kk .. + 15: 8 TMEM columns of A
+                                    const uint32_t a_tmem =
+                                        tmem + a_col + static_cast<uint32_t>((ks * kKSlice + 16 * kk) >> 1);
+                                    const uint64_t b_desc = b_k + static_cast<uint64_t>((kk * 2048) >> 4);
+                                    umma_bf16_pair_ts(d_tmem, a_tmem, b_desc, idesc, (ks | kk) ? 1u : 0u);
+                                }
+                            }
+                            issued_any = true;
+                            umma_commit_pair_mask(bar_tfull + 8 * acc.slot, both);
+                            PAIR_TRACE(k, ps + bi, j, 4);
+                            acc.next(kPairAcc);
                         }
-                        issued_any = true;
+                        if (!ok) break;
                         umma_commit_pair_mask(bar_w2_empty + 8 * w2.slot, both);
                         umma_commit_pair_mask(bar_w2_empty + 8 * w2b.slot, both);
                         w2b.next(kW2Stages);
                         w2 = w2b;
-                        umma_commit_pair_mask(bar_tfull + 8 * acc.slot, both);
-                        PAIR_TRACE(k, ps, j, 4);
-                        acc.next(kPairAcc);
                     }
                     if (!ok) break;
-                    umma_commit_pair_mask(bar_aempty + 8 * abuf, both);
+                    for (int bi = 0; bi < nb; ++bi)
+                        umma_commit_pair_mask(bar_aempty + 8 * a_buf(k, kSpMax * sp + bi), both);
                 }
             if (issued_any) {
                 umma_commit_pair(bar_drain);
@@ -543,22 +583,16 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
         }
         epi_sync512();
 
-        // this warp's share of A for pass ps of position k (launch-wide pass number P):
-        // K elements 64c .. 64c + 63 of the W1 rows of its quadrant's 32 requests (zeros for
-        // rows without a request), loaded into registers (a whole 128-byte line per lane)
-        // and stored into A buffer P mod 2 of TMEM, once the MMAs of pass P - 2 have
-        // released that buffer.  `wait` false only tests the release; the result says
-        // whether the rows were stored (false also after a failure).
-        auto gather = [&](int k, int ps, bool wait) -> bool {
-            const int P = (k - 1) * npass + ps;
-            const int abuf = P & 1;
-            const uint32_t free_parity = (static_cast<uint32_t>(P >> 1) & 1u) ^ 1u;
-            if (wait) {
-                if (!__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty + 8 * abuf, free_parity, ctl, p))) {
-                    ok = false;
-                    return false;
-                }
-            } else if (!__all_sync(0xFFFFFFFFu, mbar_test_wait(bar_aempty + 8 * abuf, free_parity))) {
+        // this warp's share of A for block ps of position k: K elements 64c .. 64c + 63 of
+        // the W1 rows of its quadrant's 32 requests (zeros for rows without a request),
+        // loaded into registers (a whole 128-byte line per lane) and stored into the block's
+        // A buffer in TMEM, once the MMAs of that buffer's previous use have released it
+        // (bounded wait).  The result says whether the rows were stored.
+        auto gather = [&](int k, int ps) -> bool {
+            const int abuf = a_buf(k, ps);
+            const uint32_t free_parity = (a_uses(k, ps) & 1u) ^ 1u;
+            if (!__all_sync(0xFFFFFFFFu, wait_bar(bar_aempty + 8 * abuf, free_parity, ctl, p))) {
+                ok = false;
                 return false;
             }
             const int tok = sh.tok[ps][row];
@@ -627,94 +661,107 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                     const int tok = sh.tok[ps][row];
                     if (tok >= 0) prefetch_l2(p.W1 + static_cast<size_t>(tok) * kRank + c * 64);
                 }
-                // the rows of the first two passes, each into its own A buffer
-                if (gather(k, 0, true) && npass > 1) gather(k, 1, true);
+                // the rows of the first super-pass's blocks, each into its own A buffer
+                if (gather(k, 0) && npass > 1) gather(k, 1);
             }
-            for (int ps = 0; ps < npass; ++ps) {
-                const int pass = (k - 1) * npass + ps;
-                const int b_row = ps * kPairRows + static_cast<int>(rank) * kRows + row;
-                const bool active = ps * kPairRows + static_cast<int>(rank) * kRows + q * 32 < p.B;
+            for (int sp = 0; sp < nsp; ++sp) {
+                const int S = (k - 1) * nsp + sp;
+                const int nb = sp_blocks(sp);
+                RowBest best[kSpMax];
+                // Gumbel-max runs one block per super-pass: its row's noise key, once
+                static_assert(!kGumbel || kSpMax == 1, "one block per super-pass with noise");
                 const RowNoise rn = kGumbel ? row_noise(static_cast<uint32_t>(k - 1),
-                                                        static_cast<uint32_t>(b_row + p.b_offset),
+                                                        static_cast<uint32_t>(sp * kPairRows + static_cast<int>(rank) * kRows +
+                                                                              row + p.b_offset),
                                                         p.seed_lo, p.seed_hi)
                                             : RowNoise{0u, 0u, 0u, 0u};
-                // the pass after next reuses this pass's A buffer: its rows go in as soon
-                // as this pass's MMAs are done with it
-                bool next_gathered = ps + 2 >= npass;
-                RowBest best;
                 for (int j = 0; j < ntiles; ++j) {
                     int first, count;
-                    tile_span(snake(pass, j, ntiles), n_units, ntiles, first, count);
+                    tile_span(snake(S, j, ntiles), n_units, ntiles, first, count);
                     const int nbox = (count + 1) >> 1;
                     const int box = c >> 1;
-                    // the U box first (it is usually there already), then the accumulator: the
-                    // chunk goes to registers and the slot is released at once, so that the
-                    // next MMAs into it overlap the arithmetic below
-                    Ring my = ur;
-                    for (int i = 0; i < box; ++i) my.next(kUSlots);
-                    const bool has_box = box < nbox;
-                    if (ok && has_box &&
-                        !__all_sync(0xFFFFFFFFu, wait_bar(bar_u_full + 8 * my.slot, my.phase, ctl, p)))
-                        ok = false;
-                    if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 12 + (warp == 12));
-                    // warp-uniform: tcgen05.ld below needs every lane of the warp
-                    if (ok && !__all_sync(0xFFFFFFFFu,
-                                          wait_bar(bar_tfull + 8 * acc.slot, acc.phase, ctl, p)))
-                        ok = false;
-                    if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 16 + (warp == 12) * 4);
-                    if (ok) {
-                        auto release = [&]() {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                if (lead) mbar_arrive(bar_tempty + 8 * acc.slot);
-                                else mbar_arrive_remote(tempty_lead + 8 * acc.slot);
-                            }
-                        };
-                        tc_fence_after();
-                        if (active && c < count) {
-                            uint32_t a[32];
-                            tmem_ld_32x32b_x32(
-                                t_lane + static_cast<uint32_t>(acc.slot * kAccCols + c * kUnit), a);
-                            tmem_wait_ld();
-                            release();
-                            if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 17 + (warp == 12) * 4);
-                            chunk_update<kGumbel>(best, a, sU + my.slot * kUSlotBytes, row, c & 1,
-                                         (u_begin + first + c) * kUnit, p, rn, c2);
-                        } else {
-                            release();
-                        }
-                        __syncwarp();
-                        if (lane == 0 && has_box) mbar_arrive(bar_u_empty + 8 * my.slot);
-                    }
-                    if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 18 + (warp == 12) * 4);
-                    for (int i = 0; i < nbox; ++i) ur.next(kUSlots);
-                    acc.next(kPairAcc);
-                    // the next pass's rows are gathered as soon as the MMAs have released A
-                    if (ok && !next_gathered && gather(k, ps + 2, false)) next_gathered = true;
-                }
-                if (ok && !next_gathered) gather(k, ps + 2, true);
-                // combine the four chunk warps of each row, one atomic per row and CTA
-                sh.part_key[c][row] = argmax_key(best.s, best.v);
-                sh.part_logit[c][row] = best.l;
-                epi_sync512();
-                if (c == 0) {
-                    unsigned long long kb = sh.part_key[0][row];
-                    float lb = sh.part_logit[0][row];
 #pragma unroll
-                    for (int i = 1; i < kChunks; ++i) {
-                        const unsigned long long ki = sh.part_key[i][row];
-                        if (ki > kb) {
-                            kb = ki;
-                            lb = sh.part_logit[i][row];
+                    for (int bi = 0; bi < kSpMax; ++bi) {
+                        if (bi >= nb) break;
+                        const int ps = kSpMax * sp + bi;
+                        const bool active = ps * kPairRows + static_cast<int>(rank) * kRows + q * 32 < p.B;
+                        // the U box first (it is usually there already), then the accumulator:
+                        // the chunk goes to registers and the slot is released at once, so that
+                        // the next MMAs into it overlap the arithmetic below
+                        Ring my = ur;
+                        for (int i = 0; i < box; ++i) my.next(kUSlots);
+                        const bool has_box = box < nbox;
+                        if (ok && has_box &&
+                            !__all_sync(0xFFFFFFFFu, wait_bar(bar_u_full + 8 * my.slot, my.phase, ctl, p)))
+                            ok = false;
+                        if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 12 + (warp == 12));
+                        // warp-uniform: tcgen05.ld below needs every lane of the warp
+                        if (ok && !__all_sync(0xFFFFFFFFu,
+                                              wait_bar(bar_tfull + 8 * acc.slot, acc.phase, ctl, p)))
+                            ok = false;
+                        if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 16 + (warp == 12) * 4);
+                        if (ok) {
+                            auto release = [&]() {
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) {
+                                    if (lead) mbar_arrive(bar_tempty + 8 * acc.slot);
+                                    else mbar_arrive_remote(tempty_lead + 8 * acc.slot);
+                                }
+                            };
+                            tc_fence_after();
+                            if (active && c < count) {
+                                uint32_t a[32];
+                                tmem_ld_32x32b_x32(
+                                    t_lane + static_cast<uint32_t>(acc.slot * kAccCols + c * kUnit), a);
+                                tmem_wait_ld();
+                                release();
+                                if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 17 + (warp == 12) * 4);
+                                chunk_update<kGumbel>(best[bi], a, sU + my.slot * kUSlotBytes, row, c & 1,
+                                                      (u_begin + first + c) * kUnit, p, rn, c2);
+                            } else {
+                                release();
+                            }
+                            __syncwarp();
+                            if (lane == 0 && has_box) mbar_arrive(bar_u_empty + 8 * my.slot);
                         }
+                        if (lane == 0 && (warp == 0 || warp == 12)) PAIR_TRACE(k, ps, j, 18 + (warp == 12) * 4);
+                        for (int i = 0; i < nbox; ++i) ur.next(kUSlots);
+                        acc.next(kPairAcc);
                     }
-                    sh.cta_key[ps][row] = kb;
-                    sh.cta_logit[ps][row] = lb;
-                    if (ok && b_row < p.B)
-                        atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + b_row], kb);
                 }
-                epi_sync512();
+                // combine the four chunk warps of each row, one atomic per row and CTA, block
+                // by block
+#pragma unroll
+                for (int bi = 0; bi < kSpMax; ++bi) {
+                    if (bi >= nb) break;
+                    const int ps = kSpMax * sp + bi;
+                    const int b_row = ps * kPairRows + static_cast<int>(rank) * kRows + row;
+                    sh.part_key[c][row] = argmax_key(best[bi].s, best[bi].v);
+                    sh.part_logit[c][row] = best[bi].l;
+                    epi_sync512();
+                    if (c == 0) {
+                        unsigned long long kb = sh.part_key[0][row];
+                        float lb = sh.part_logit[0][row];
+#pragma unroll
+                        for (int i = 1; i < kChunks; ++i) {
+                            const unsigned long long ki = sh.part_key[i][row];
+                            if (ki > kb) {
+                                kb = ki;
+                                lb = sh.part_logit[i][row];
+                            }
+                        }
+                        sh.cta_key[ps][row] = kb;
+                        sh.cta_logit[ps][row] = lb;
+                        if (ok && b_row < p.B)
+                            atomicMax(&p.slots[static_cast<size_t>(k - 1) * p.B + b_row], kb);
+                    }
+                    epi_sync512();
+                }
+                // the blocks that reuse this super-pass's A buffers (blocks 0 and 1 went in at
+                // the position's start), once its MMAs have released them
+                for (int ps = kSpMax * sp + 2; ps < kSpMax * sp + kSpMax + 2 && ps < npass; ++ps)
+                    if (ok) gather(k, ps);
             }
 
             // ---- grid barrier: every CTA has combined its rows of position k
@@ -739,10 +786,11 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
         }
         // the last pair commit on aempty may still be arriving on this CTA's barrier
         if (ok) {
-            const int passes = p.gamma * npass;
             for (int b = 0; b < kABufs; ++b) {
-                const int uses = (passes + 1 - b) / 2;     // passes P < passes with P mod 2 = b
-                if (uses > 0) wait_drain(bar_aempty + 8 * b, static_cast<uint32_t>(uses - 1) & 1u, p);
+                // uses over the launch: the count before block b of a position past the last
+                const uint32_t uses = kSpMax == 2 ? (b < npass ? abuf_uses(p.gamma + 1, b, npass) : 0u)
+                                                  : static_cast<uint32_t>((p.gamma * npass + 1 - b) / 2);
+                if (uses > 0) wait_drain(bar_aempty + 8 * b, (uses - 1) & 1u, p);
             }
         }
     }
