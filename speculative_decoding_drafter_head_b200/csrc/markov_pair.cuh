@@ -488,14 +488,9 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                 for (int sp = 0; sp < nsp && ok; ++sp) {
                     const int S = (k - 1) * nsp + sp;
                     const int nb = sp_blocks(sp);
-                    // block ps = kSpMax sp + bi reads A buffer ps mod 2
-                    for (int bi = 0; bi < nb && ok; ++bi) {
-                        const int ps = kSpMax * sp + bi;
-                        if (!wait_bar(bar_afull + 8 * a_buf(k, ps), a_uses(k, ps) & 1u, ctl, p))
-                            ok = false;
-                    }
-                    if (!ok) break;
-                    tc_fence_after();
+                    // block ps = kSpMax sp + bi reads A buffer ps mod 2; its rows are waited
+                    // for right before its first MMAs (the first tile's), so that block 0's
+                    // MMAs start while block 1's rows are still being gathered
                     for (int j = 0; j < ntiles && ok; ++j) {
                         [[maybe_unused]] const int ps = kSpMax * sp;
                         int first, count;
@@ -524,6 +519,11 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
                                 break;
                             }
                             PAIR_TRACE(k, ps + bi, j, 2);
+                            if (j == 0 && !wait_bar(bar_afull + 8 * a_buf(k, ps + bi),
+                                                    a_uses(k, ps + bi) & 1u, ctl, p)) {
+                                ok = false;
+                                break;
+                            }
                             tc_fence_after();
                             const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc.slot * kAccCols);
                             const uint32_t a_col = kACol + static_cast<uint32_t>(a_buf(k, ps + bi) * kAccCols);
