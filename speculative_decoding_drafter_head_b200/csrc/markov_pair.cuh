@@ -15,9 +15,11 @@
 // that the next block's rows are in place before its first MMA and the tensor core reads
 // only W2 from shared memory, whose bandwidth the TMA copies and the epilogue's U reads
 // share.  Each pair owns a contiguous vocabulary slice cut into 128-column tiles; for
-// every position k and every block of 256 requests (a pass) it walks the tiles,
-// alternating direction from one pass to the next, so that the tiles read last are read
-// again first and are still in L2.
+// every position k it walks the tiles once per super-pass, alternating direction from
+// one walk to the next, so that the tiles read last are read again first and are still
+// in L2.  In greedy drafting a super-pass is two blocks of 256 requests: every W2 tile
+// then feeds 16 MMAs per block (one accumulator each) before its stages are released.
+// Gumbel-max, bound by its selection arithmetic, walks once per block.
 //
 // Per CTA: 16 epilogue warps (four per TMEM lane quadrant, one 32-column chunk of every
 // tile each), warp 16 the W2 producer (TMA, 64 columns x 128 K rows per stage), warp 17
@@ -47,7 +49,7 @@ constexpr int kWarpW2 = kEpiWarps, kWarpU = kEpiWarps + 1, kWarpMma = kEpiWarps 
 constexpr int kThreads = (kEpiWarps + 3) * 32;        // 608
 constexpr int kWarpConfPair = kEpiWarps + 3;          // confidence head (kConf instances)
 constexpr int kThreadsConfPair = kThreads + 32;       // 640
-constexpr int kRows = 128;                            // requests per CTA per pass
+constexpr int kRows = 128;                            // requests per CTA per block
 constexpr int kPairRows = 2 * kRows;                  // the pair MMA's M
 constexpr int kW2Stages = 7;
 constexpr int kW2StageBytes = 64 * kKSlice * 2;       // 64 columns x 128 K rows: 16 KB
@@ -56,7 +58,7 @@ constexpr int kUSlotBytes = kRows * kUBoxCols * 2;    // 128 rows x 64 columns: 
 constexpr int kDynSmem = kW2Stages * kW2StageBytes + kUSlots * kUSlotBytes + 1024;
 // TMEM (512 columns): two 128-column accumulators, then two buffers of A = W1[x_{k-1}]
 // for the CTA's 128 rows (row m in lane m, K = 256 bf16 packed two per column: 128
-// columns each), so that the next pass's rows are in place before its first MMA
+// columns each): one per block of a super-pass
 constexpr int kPairAcc = 2;
 constexpr int kABufs = 2;
 constexpr uint32_t kACol = kPairAcc * kAccCols;       // 256: A buffer b at 256 + 128 b
@@ -85,13 +87,13 @@ struct Shared {
     Ctl ctl;
     unsigned long long part_key[kChunks][kRows];   // per chunk warp, before the CTA combine
     float part_logit[kChunks][kRows];
-    unsigned long long cta_key[kMaxPasses][kRows];  // this CTA's best per row and pass
+    unsigned long long cta_key[kMaxPasses][kRows];  // this CTA's best per row and block
     float cta_logit[kMaxPasses][kRows];
     int tok[kMaxPasses][kRows];                     // x_{k-1} of this CTA's rows (-1: none)
     int go;                                         // verdict of the last grid barrier
 };
 
-// Optional per-tile timeline (build with -DDSPARK_TRACE): for position 2, pass 0, tile j
+// Optional per-tile timeline (build with -DDSPARK_TRACE): for position 2, block 0, tile j
 // and event e, a %globaltimer stamp in g_trace[(blockIdx.x * 64 + j) * 32 + e].
 #ifdef DSPARK_TRACE
 #define PAIR_TRACE(k, ps, j, e)                                                               \
@@ -656,7 +658,7 @@ __global__ void __launch_bounds__(kConf ? kThreadsConfPair : kThreads, 1)
 
         for (int k = 1; k <= p.gamma; ++k) {
             if (ok) {
-                // L2 prefetch of the W1 lines the later passes of this position will gather
+                // L2 prefetch of the W1 lines the later blocks of this position will gather
                 for (int ps = 1; ps < npass; ++ps) {
                     const int tok = sh.tok[ps][row];
                     if (tok >= 0) prefetch_l2(p.W1 + static_cast<size_t>(tok) * kRank + c * 64);
