@@ -204,6 +204,12 @@ STRESS = [
     synth.Workload("stress B=3 gamma=64 V=2048", B=3, gamma=64, V=2048, d=64, w_std=0.3, seed=4),
     synth.Workload("stress B=130 gamma=64 V=1032", B=130, gamma=64, V=1032, d=64, w_std=0.3,
                    seed=6),
+    # pair kernel: Gumbel-max over three 256-request blocks (one block per walk, the block
+    # after next gathered into the buffer just released), and greedy over four blocks, two
+    # per W2 tile, the last one partial (232 rows)
+    synth.Workload("stress B=600 V=3000 gumbel", B=600, gamma=3, V=3000, d=64, w_std=0.2,
+                   logits="zipf", mode=1, tau=0.7, seed=9),
+    synth.Workload("stress B=1000 V=2056", B=1000, gamma=3, V=2056, d=64, w_std=0.2, seed=10),
 ]
 
 
